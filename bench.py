@@ -1,0 +1,383 @@
+"""Benchmark of split-KV tail-padded attention on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload cosmos_self]
+
+A step is one call of attn_fwd_split_kv over one batch of the workload (the
+whole hot path: one kernel).  Inputs are synthetic (seeded, see workloads/)
+and rotate over 4 device copies (> 126 MB L2) so no step reads another step's
+data from L2.  Device time is measured with CUDA events on the launching
+stream, W warm-up steps first, barrier + synchronize on both sides, max over
+ranks.  N > 1 (torchrun) runs one independent copy of the workload per rank
+(weak scaling, no collective on the data path).
+
+--impl reference times the CPU oracle (the slow, obviously-correct fp64
+definition) on the host cores, each step a bounded sample of query rows of
+the same workload, reported in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "split-KV attention TFLOP/s and % of B200 dense-bf16 peak; max-abs err vs CPU oracle"
+DEFAULT_WORKLOAD = "cosmos_self"
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["varlen_flash_attention_b200/csrc/attn_fwd_sm100.cuh",
+                  "varlen_flash_attention_b200/csrc/ptx.cuh",
+                  "varlen_flash_attention_b200/csrc/splitkv_attn.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def q_valid_of(w):
+    rl = w.real_lens()
+    return list(rl) if w.Sq == w.Skv else [w.Sq] * w.B
+
+
+def flops_of(w, rows=None):
+    """Algorithmic FLOPs: 4 * D * Hq * sum_b (valid query rows) * real_len[b]."""
+    rl = w.real_lens()
+    qv = q_valid_of(w)
+    if rows is not None:
+        qv = [sum(1 for r in rows if r < qv[b]) for b in range(w.B)]
+    return 4.0 * w.D * w.Hq * sum(q * n for q, n in zip(qv, rl))
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def traffic_per_launch(workload):
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, clock-event reasons) from a thread while running."""
+
+    REASONS = {
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:  # no NVML: clocks reported as unavailable
+            self._ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS.items():
+                    if r & getattr(nv, attr, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.0005)
+
+    def __enter__(self):
+        if self._ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self.t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return rank, world, local, dist
+    return 0, 1, 0, None
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(x, dist):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, dist):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def cpu_oracle_sample(w, target_s=10.0, seed=0):
+    """Time the fp64 oracle on a bounded row sample of the workload (host cores)."""
+    import numpy as np
+
+    import oracle
+
+    t = workloads.make_inputs(w)
+    rl = w.real_lens()
+    rng = np.random.default_rng(seed)
+    n = max(1, min(w.Sq, 16))
+    rows = sorted(int(r) for r in rng.choice(w.Sq, size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_split_kv(**t, real_len=rl, rows=rows)
+    dt = time.perf_counter() - t0
+    n2 = int(min(w.Sq, max(n, n * target_s / max(dt, 1e-3))))
+    rows = sorted(int(r) for r in rng.choice(w.Sq, size=n2, replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_split_kv(**t, real_len=rl, rows=rows)
+    dt = time.perf_counter() - t0
+    fl = flops_of(w, rows)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} of {w.Sq} query rows x {w.Hq} heads x {w.B} batch rows of {w.name} "
+                      f"({fl / 1e9:.1f} GFLOP, {dt:.1f} s)"}
+
+
+def run_reference(args, w):
+    """The CPU oracle as the reference arm: each step a bounded row sample."""
+    import numpy as np
+
+    import oracle
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    t = workloads.make_inputs(w)
+    rl = w.real_lens()
+    rng = np.random.default_rng(1)
+    # about 3 s of CPU work per step at this machine's oracle speed
+    probe = sorted(int(r) for r in rng.choice(w.Sq, size=min(w.Sq, 8), replace=False))
+    t0 = time.perf_counter()
+    oracle.attn_split_kv(**t, real_len=rl, rows=probe)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    per_step = int(min(w.Sq, max(1, len(probe) * 3.0 / dt)))
+    samples = [sorted(int(r) for r in rng.choice(w.Sq, size=per_step, replace=False))
+               for _ in range(args.warmup + args.steps)]
+    for rows in samples[: args.warmup]:
+        oracle.attn_split_kv(**t, real_len=rl, rows=rows)
+    fl = 0.0
+    t0 = time.perf_counter()
+    for rows in samples[args.warmup:]:
+        oracle.attn_split_kv(**t, real_len=rl, rows=rows)
+        fl += flops_of(w, rows)
+    dt = time.perf_counter() - t0
+    value = fl / dt / 1e12
+    sample = f"{per_step} of {w.Sq} query rows x {w.Hq} heads x {w.B} batch rows of {w.name} per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.B, "seq_q": w.Sq, "prefix": w.Sp, "suffix": w.Ss,
+                   "real_len": rl, "heads_q": w.Hq, "heads_kv": w.Hkv, "head_dim": w.D},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    import varlen_flash_attention_b200 as sk
+
+    rank, world, local, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    rl = w.real_lens()
+    n_copies = 4
+    host = workloads.make_inputs(w, seed=w.seed + 1000 * rank)
+    keys = ("q", "k_prefix", "v_prefix", "k_suffix", "v_suffix")
+    copies = [{k: host[k].to(dev) for k in keys} for _ in range(n_copies)]
+    outs = [torch.empty(w.B, w.Sq, w.Hq, w.D, dtype=torch.bfloat16, device=dev) for _ in range(n_copies)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        c = copies[i % n_copies]
+        sk.attn_fwd_split_kv(c["q"], c["k_prefix"], c["v_prefix"], c["k_suffix"], c["v_suffix"],
+                             real_len=rl, out=outs[i % n_copies], stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    sk.sk_device_status(local, clear=True)
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(dist)
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dist)
+    dt_ms = ev0.elapsed_time(ev1)
+    status = sk.sk_device_status(local, clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    dt_ms_max = max_over_ranks(dt_ms, dist)
+    fl = flops_of(w)
+    value = sum_over_ranks(fl * args.steps, dist) / (dt_ms_max / 1e3) / 1e12
+    per_launch_ms = dt_ms / args.steps
+    achieved = fl / (per_launch_ms / 1e3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), H2D + kernel + D2H
+    pinned = {k: host[k].pin_memory() for k in keys}
+    out_host = torch.empty(w.B, w.Sq, w.Hq, w.D, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(pinned[k].numel() * 2 for k in keys)
+    d2h = out_host.numel() * 2
+    dbuf = {k: torch.empty_like(copies[0][k]) for k in keys}
+    dout = torch.empty_like(outs[0])
+
+    def e2e_step():
+        for k in keys:
+            dbuf[k].copy_(pinned[k], non_blocking=True)
+        sk.attn_fwd_split_kv(dbuf["q"], dbuf["k_prefix"], dbuf["v_prefix"], dbuf["k_suffix"],
+                             dbuf["v_suffix"], real_len=rl, out=dout, stream=stream)
+        out_host.copy_(dout, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dist)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist)
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist)
+    e2e_value = sum_over_ranks(fl * args.steps, dist) / (e2e_ms / 1e3) / 1e12
+
+    peak, peak_kind = measured_peaks()
+    clocks = clk.summary()
+    line = None
+    if rank == 0:
+        cpu = cpu_oracle_sample(w) if world == 1 and not args.no_cpu_baseline else None
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": dt_ms_max / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.B, "seq_q": w.Sq, "prefix": w.Sp, "suffix": w.Ss,
+                       "real_len": rl, "heads_q": w.Hq, "heads_kv": w.Hkv, "head_dim": w.D,
+                       "flop_per_step": fl, "l2": "inputs rotate over 4 device copies (> 126 MB L2)",
+                       "parallelism": f"replica x{world}" if world > 1 else "single"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_kind": f"{peak_kind} bf16 burst",
+                         "traffic": traffic_per_launch(w.name)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = workloads.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

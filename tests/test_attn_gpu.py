@@ -1,0 +1,311 @@
+"""Parity of the sm_100a split-KV attention kernel (through the C ABI) with the
+fp64 CPU oracle, on the same seeded inputs.
+
+Bar (the workload contract): bf16 output vs fp64 oracle, max-abs <= 2e-2 and
+relative L2 <= 1e-2; exact agreement on which rows/keys are valid: pad query
+rows must be exactly 0, and results must not change (bitwise) when pad
+contents change.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_L2 = 1e-2
+
+
+@pytest.fixture(scope="module")
+def sk():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from varlen_flash_attention_b200 import build
+
+    build.build()
+    import varlen_flash_attention_b200 as m
+
+    return m
+
+
+def _to_dev(t):
+    return {k: v.cuda() for k, v in t.items()}
+
+
+def _compare(got, ref, what=""):
+    got = got.astype(np.float64)
+    diff = np.abs(got - ref)
+    max_abs = float(diff.max()) if diff.size else 0.0
+    denom = float(np.sqrt((ref ** 2).sum()))
+    rel = float(np.sqrt((diff ** 2).sum()) / denom) if denom > 0 else max_abs
+    assert np.all(np.isfinite(got)), what
+    assert max_abs <= MAX_ABS, f"{what} max_abs={max_abs}"
+    assert rel <= REL_L2, f"{what} rel_l2={rel}"
+    return max_abs, rel
+
+
+def _run(sk, t, real_len=None, q_valid=None, scale=None):
+    d = _to_dev(t)
+    out = sk.attn_fwd_split_kv(d["q"], d["k_prefix"], d["v_prefix"], d["k_suffix"], d["v_suffix"],
+                               real_len=real_len, q_valid=q_valid, softmax_scale=scale)
+    torch.cuda.synchronize()
+    return out
+
+
+def _check_case(sk, t, real_len=None, q_valid=None, scale=None, rows=None, what=""):
+    out = _run(sk, t, real_len, q_valid, scale).float().cpu().numpy()
+    ref = oracle.attn_split_kv(**t, real_len=real_len, q_valid=q_valid, softmax_scale=scale, rows=rows)
+    got = out if rows is None else out[:, rows]
+    B, Sq = t["q"].shape[:2]
+    Skv = t["k_prefix"].shape[1] + t["k_suffix"].shape[1]
+    rl = real_len if real_len is not None else [Skv] * B
+    qv = q_valid if q_valid is not None else oracle.q_valid_rule(Sq, Skv, rl)
+    # exact zeros for pad rows / rows without a valid key
+    for b in range(B):
+        if rl[b] == 0:
+            assert np.all(out[b] == 0.0), what
+        assert np.all(out[b, qv[b]:] == 0.0), what
+    return _compare(got, ref, what)
+
+
+# ---------------------------------------------------------------- the five workloads
+
+
+def test_tiny_workload(sk):
+    w = workloads.get("tiny")
+    _check_case(sk, workloads.make_inputs(w), what="tiny")
+
+
+def _sample_rows(Sq, n, seed, forced=()):
+    g = np.random.default_rng(seed)
+    rows = set(int(r) for r in g.choice(Sq, size=min(n, Sq), replace=False))
+    rows.update(r for r in forced if 0 <= r < Sq)
+    return sorted(rows)
+
+
+def test_cosmos_self_attention(sk):
+    w = workloads.get("cosmos_self")
+    t = workloads.make_inputs(w)
+    rows = _sample_rows(w.Sq, 192, 1, forced=(0, 127, 128, 4095))
+    _check_case(sk, t, rows=rows, what="cosmos_self")
+
+
+def test_tail_padded_joint(sk):
+    w = workloads.get("tail_padded_joint")
+    t = workloads.make_inputs(w)
+    rows = _sample_rows(w.Sq, 160, 2, forced=(0, 4351, 4352, 4428, 4429, 4430, 4431))
+    _check_case(sk, t, real_len=w.real_lens(), rows=rows, what="tail_padded_joint")
+
+
+def test_cross_short_kv(sk):
+    w = workloads.get("cross_short_kv")
+    t = workloads.make_inputs(w)
+    rows = _sample_rows(w.Sq, 384, 3, forced=(0, 32759, 32639, 32640))
+    _check_case(sk, t, rows=rows, what="cross_short_kv")
+
+
+def test_long_gqa(sk):
+    w = workloads.get("long_gqa")
+    t = workloads.make_inputs(w)
+    forced = (0, 511, 512, 25047) + tuple(range(25048, 25088))
+    rows = _sample_rows(w.Sq, 96, 5, forced=forced)
+    _check_case(sk, t, real_len=w.real_lens(), rows=rows, what="long_gqa")
+
+
+# ---------------------------------------------------------------- random shapes, edges
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_shapes(sk, seed):
+    gen = torch.Generator().manual_seed(1000 + seed)
+    D = [64, 128][seed % 2]
+    w = workloads.random_workload(gen, D=D, max_sq=400, max_skv=700)
+    t = workloads.make_inputs(w)
+    _check_case(sk, t, real_len=w.real_lens(), what=f"random{seed}")
+
+
+@pytest.mark.parametrize("Sp,Ss,rl", [
+    (0, 300, 300), (300, 0, 300), (128, 128, 256), (129, 127, 256), (16, 64, 80),
+    (200, 200, 150), (200, 200, 0), (1, 1, 1), (127, 1, 128), (130, 500, 129),
+])
+def test_split_points_and_clipping(sk, Sp, Ss, rl):
+    gen = torch.Generator().manual_seed(Sp * 1000 + Ss)
+    D, Hq, Hkv, Sq = 128, 4, 2, 200
+    t = {
+        "q": torch.randn(2, Sq, Hq, D, generator=gen).to(torch.bfloat16),
+        "k_prefix": torch.randn(2, Sp, Hkv, D, generator=gen).to(torch.bfloat16),
+        "v_prefix": torch.randn(2, Sp, Hkv, D, generator=gen).to(torch.bfloat16),
+        "k_suffix": torch.randn(2, Ss, Hkv, D, generator=gen).to(torch.bfloat16),
+        "v_suffix": torch.randn(2, Ss, Hkv, D, generator=gen).to(torch.bfloat16),
+    }
+    _check_case(sk, t, real_len=[rl, Sp + Ss], what=f"split {Sp}+{Ss} rl={rl}")
+
+
+def test_split_invariance_against_oracle(sk):
+    """Every split point of the same keys gives the oracle's (split-free) result."""
+    gen = torch.Generator().manual_seed(77)
+    D, H, Sq, Skv = 128, 2, 256, 700
+    q = torch.randn(1, Sq, H, D, generator=gen).to(torch.bfloat16)
+    k = torch.randn(1, Skv, H, D, generator=gen).to(torch.bfloat16)
+    v = torch.randn(1, Skv, H, D, generator=gen).to(torch.bfloat16)
+    ref = oracle.attn_split_kv(q, k[:, :0], v[:, :0], k, v, real_len=[650])
+    for p in (0, 1, 127, 128, 129, 512, 650, 700):
+        t = dict(q=q, k_prefix=k[:, :p].contiguous(), v_prefix=v[:, :p].contiguous(),
+                 k_suffix=k[:, p:].contiguous(), v_suffix=v[:, p:].contiguous())
+        out = _run(sk, t, real_len=[650]).float().cpu().numpy()
+        _compare(out, ref, f"split p={p}")
+
+
+@pytest.mark.parametrize("fill", [float("nan"), float("inf"), 1e4])
+def test_pad_contents_never_matter_bitwise(sk, fill):
+    w = workloads.get("tail_padded_joint")
+    t = workloads.make_inputs(w)
+    rl = w.real_lens()
+    base = _run(sk, t, real_len=rl)
+    poisoned = workloads.poison_pad(t, w.Sp, rl, oracle.q_valid_rule(w.Sq, w.Skv, rl), fill)
+    got = _run(sk, poisoned, real_len=rl)
+    assert torch.equal(base.view(torch.int16), got.view(torch.int16))
+
+
+def test_pad_invariance_appending_pad(sk):
+    """Appending tail pad to an unpadded problem changes no real row (bitwise)."""
+    gen = torch.Generator().manual_seed(3)
+    D, H, Sp, Ss = 128, 2, 100, 300
+    q = torch.randn(1, Sp + Ss, H, D, generator=gen).to(torch.bfloat16)
+    kp, vp = (torch.randn(1, Sp, H, D, generator=gen).to(torch.bfloat16) for _ in range(2))
+    ks, vs = (torch.randn(1, Ss, H, D, generator=gen).to(torch.bfloat16) for _ in range(2))
+    base = _run(sk, dict(q=q, k_prefix=kp, v_prefix=vp, k_suffix=ks, v_suffix=vs))
+    for npad in (1, 40, 200):
+        nan = torch.full((1, npad, H, D), float("nan"), dtype=torch.bfloat16)
+        got = _run(sk, dict(q=torch.cat([q, nan], 1), k_prefix=kp, v_prefix=vp,
+                            k_suffix=torch.cat([ks, nan], 1), v_suffix=torch.cat([vs, nan], 1)),
+                   real_len=[Sp + Ss])
+        assert torch.equal(got[:, : Sp + Ss].view(torch.int16), base.view(torch.int16))
+        assert torch.all(got[:, Sp + Ss:] == 0)
+
+
+def test_uniform_v_gives_one(sk):
+    gen = torch.Generator().manual_seed(4)
+    q = (torch.randn(1, 300, 2, 128, generator=gen) * 3).to(torch.bfloat16)
+    kp = (torch.randn(1, 40, 2, 128, generator=gen) * 3).to(torch.bfloat16)
+    ks = (torch.randn(1, 500, 2, 128, generator=gen) * 3).to(torch.bfloat16)
+    out = _run(sk, dict(q=q, k_prefix=kp, v_prefix=torch.ones_like(kp), k_suffix=ks,
+                        v_suffix=torch.ones_like(ks)), real_len=[511])
+    assert float((out.float() - 1).abs().max()) <= 2.0 ** -7
+
+
+def test_gqa_head_mapping(sk):
+    gen = torch.Generator().manual_seed(5)
+    Hq, Hkv, D = 32, 8, 128
+    g = Hq // Hkv
+    q = torch.randn(1, 130, Hq, D, generator=gen).to(torch.bfloat16)
+    kp = torch.randn(1, 64, Hkv, D, generator=gen).to(torch.bfloat16)
+    ks = torch.randn(1, 200, Hkv, D, generator=gen).to(torch.bfloat16)
+    vp = torch.empty(1, 64, Hkv, D, dtype=torch.bfloat16)
+    vs = torch.empty(1, 200, Hkv, D, dtype=torch.bfloat16)
+    for h in range(Hkv):
+        vp[:, :, h] = h + 1
+        vs[:, :, h] = h + 1
+    out = _run(sk, dict(q=q, k_prefix=kp, v_prefix=vp, k_suffix=ks, v_suffix=vs)).float().cpu()
+    for hq in range(Hq):
+        assert torch.allclose(out[0, :, hq], torch.full_like(out[0, :, hq], hq // g + 1), atol=0.02), hq
+
+
+def test_one_valid_key(sk):
+    gen = torch.Generator().manual_seed(6)
+    q = torch.randn(1, 50, 2, 64, generator=gen).to(torch.bfloat16)
+    kp = torch.randn(1, 10, 2, 64, generator=gen).to(torch.bfloat16)
+    vp = torch.randn(1, 10, 2, 64, generator=gen).to(torch.bfloat16)
+    ks = torch.randn(1, 20, 2, 64, generator=gen).to(torch.bfloat16)
+    vs = torch.randn(1, 20, 2, 64, generator=gen).to(torch.bfloat16)
+    out = _run(sk, dict(q=q, k_prefix=kp, v_prefix=vp, k_suffix=ks, v_suffix=vs), real_len=[1]).cpu()
+    for h in range(2):
+        assert torch.equal(out[0, :, h].view(torch.int16), vp[0, 0, h].expand(50, 64).view(torch.int16))
+
+
+def test_explicit_q_valid_and_empty_rows(sk):
+    gen = torch.Generator().manual_seed(7)
+    t = {k: torch.randn(3, n, 2, 128, generator=gen).to(torch.bfloat16)
+         for k, n in (("q", 300), ("k_prefix", 50), ("v_prefix", 50), ("k_suffix", 250), ("v_suffix", 250))}
+    _check_case(sk, t, real_len=[300, 0, 17], q_valid=[129, 300, 0], what="q_valid")
+
+
+def test_many_batch_rows_cross_launch_chunks(sk):
+    gen = torch.Generator().manual_seed(8)
+    B = 19
+    t = {k: torch.randn(B, n, 2, 64, generator=gen).to(torch.bfloat16)
+         for k, n in (("q", 70), ("k_prefix", 20), ("v_prefix", 20), ("k_suffix", 100), ("v_suffix", 100))}
+    rl = [(13 * b) % 121 for b in range(B)]
+    _check_case(sk, t, real_len=rl, what="B=19")
+
+
+def test_fused_qkv_strided_views_match_contiguous(sk):
+    """q/k/v as views of one [B, S, Hq + 2Hkv, D] projection (view + slice, no copy)."""
+    gen = torch.Generator().manual_seed(9)
+    B, S, Hq, Hkv, D, Sp = 2, 333, 8, 2, 128, 77
+    qkv = torch.randn(B, S, Hq + 2 * Hkv, D, generator=gen).to(torch.bfloat16).cuda()
+    q, k, v = qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:]
+    kp = torch.randn(B, Sp, Hkv, D, generator=gen).to(torch.bfloat16).cuda()
+    vp = torch.randn(B, Sp, Hkv, D, generator=gen).to(torch.bfloat16).cuda()
+    a = sk.attn_fwd_split_kv(q, kp, vp, k, v, real_len=[Sp + S, Sp + 300])
+    b = sk.attn_fwd_split_kv(q.contiguous(), kp, vp, k.contiguous(), v.contiguous(),
+                             real_len=[Sp + S, Sp + 300])
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    ref = oracle.attn_split_kv(q.cpu(), kp.cpu(), vp.cpu(), k.cpu(), v.cpu(), real_len=[Sp + S, Sp + 300])
+    _compare(a.float().cpu().numpy(), ref, "fused view")
+
+
+def test_output_canaries_untouched(sk):
+    gen = torch.Generator().manual_seed(10)
+    B, Sq, H, D = 1, 200, 2, 128
+    t = {k: torch.randn(B, n, H, D, generator=gen).to(torch.bfloat16)
+         for k, n in (("q", Sq), ("k_prefix", 30), ("v_prefix", 30), ("k_suffix", 170), ("v_suffix", 170))}
+    d = _to_dev(t)
+    pad = 32768  # 64 KB of canary on each side
+    n = B * Sq * H * D
+    buf = torch.full((pad + n + pad,), 12345, dtype=torch.int16, device="cuda")
+    out = buf[pad:pad + n].view(torch.bfloat16).view(B, Sq, H, D)
+    sk.attn_fwd_split_kv(d["q"], d["k_prefix"], d["v_prefix"], d["k_suffix"], d["v_suffix"],
+                         real_len=[150], out=out)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:pad] == 12345) and torch.all(buf[pad + n:] == 12345)
+    # Sq == Sp + Ss here, so rows >= 150 are pad and must come back as zeros
+    assert torch.all(out[:, 150:] == 0)
+    ref = oracle.attn_split_kv(**t, real_len=[150])
+    _compare(out.float().cpu().numpy(), ref, "canary")
+
+
+def test_output_written_into_strided_view(sk):
+    gen = torch.Generator().manual_seed(11)
+    B, Sq, H, D = 2, 140, 4, 64
+    t = {k: torch.randn(B, n, H, D, generator=gen).to(torch.bfloat16)
+         for k, n in (("q", Sq), ("k_prefix", 8), ("v_prefix", 8), ("k_suffix", 132), ("v_suffix", 132))}
+    d = _to_dev(t)
+    big = torch.full((B, Sq, 2 * H, D), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = big[:, :, H:]
+    sk.attn_fwd_split_kv(d["q"], d["k_prefix"], d["v_prefix"], d["k_suffix"], d["v_suffix"], out=out)
+    torch.cuda.synchronize()
+    assert torch.all(big[:, :, :H] == 7.0)
+    ref = oracle.attn_split_kv(**t)
+    _compare(out.float().cpu().numpy(), ref, "strided out")
+
+
+def test_rejections_raise(sk):
+    q = torch.zeros(1, 64, 3, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 64, 2, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sk.SplitKVError) as e:
+        sk.attn_fwd_split_kv(q, k, k, k, k)
+    assert e.value.status == 1
+    q = torch.zeros(1, 64, 2, 96, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 64, 2, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sk.SplitKVError) as e:
+        sk.attn_fwd_split_kv(q, k, k, k, k)
+    assert e.value.status == 2
+
+
+def test_device_status_clean_after_runs(sk):
+    assert sk.sk_device_status(clear=True) == 0

@@ -1,0 +1,165 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+symbol include/splitkv_attn.h declares, and rejects bad arguments before any
+CUDA call (so these run on CPU-only machines).  Every call here uses invalid
+arguments, so nothing is ever launched, on any machine."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import varlen_flash_attention_b200 as sk
+from varlen_flash_attention_b200 import SkTensor, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "splitkv_attn.h")
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return sk.lib()
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"SK_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = set(_declared_symbols())
+    assert {"attn_fwd_split_kv", "attn_fwd_split_kv_ex", "qk_rmsnorm_rope", "sk_last_error",
+            "sk_device_status", "sk_set_wait_timeout_ms", "sk_abi_version"} <= names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_abi_version(L):
+    assert sk.sk_abi_version() == 1
+
+
+def _t(len_s, sb, ss, sh, ptr=FAKE):
+    return SkTensor(ptr, sb, ss, sh, len_s)
+
+
+def _call(L, q, kp, vp, ks, vs, out, Hq=2, Hkv=2, D=64, B=1, scale=0.125, real_len=None, q_valid=None):
+    rl = (ctypes.c_int32 * B)(*real_len) if real_len is not None else None
+    args = [ctypes.byref(x) for x in (q, kp, vp, ks, vs)] + [
+        ctypes.cast(rl, ctypes.c_void_p) if rl is not None else None, Hq, Hkv, scale,
+        ctypes.byref(out), B, D]
+    if q_valid is None:
+        return L.attn_fwd_split_kv(*args, None)
+    qv = (ctypes.c_int32 * B)(*q_valid)
+    return L.attn_fwd_split_kv_ex(*args, ctypes.cast(qv, ctypes.c_void_p), None)
+
+
+def _good(D=64, H=2, Sq=64, Sp=16, Ss=64):
+    """Descriptors of a valid contiguous problem on fake, disjoint addresses."""
+    q = _t(Sq, Sq * H * D, H * D, D, FAKE)
+    kp = _t(Sp, Sp * H * D, H * D, D, FAKE + (1 << 24))
+    vp = _t(Sp, Sp * H * D, H * D, D, FAKE + (2 << 24))
+    ks = _t(Ss, Ss * H * D, H * D, D, FAKE + (3 << 24))
+    vs = _t(Ss, Ss * H * D, H * D, D, FAKE + (4 << 24))
+    out = _t(Sq, Sq * H * D, H * D, D, FAKE + (5 << 24))
+    return [q, kp, vp, ks, vs, out]
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+def _expect(L, status, *args, **kw):
+    st = _call(L, *args, **kw)
+    assert st == status, (st, L.sk_last_error())
+    assert L.sk_last_error()
+
+
+def test_rejects_gqa_indivisible(L):
+    _expect(L, INVALID, *_good(), Hq=3, Hkv=2)
+
+
+def test_rejects_unsupported_head_dim(L):
+    _expect(L, UNSUPPORTED, *_good(D=96), D=96)
+
+
+def test_rejects_misaligned_pointer(L):
+    g = _good()
+    g[0] = _t(64, 64 * 128, 128, 64, FAKE + 2)
+    _expect(L, INVALID, *g)
+
+
+def test_rejects_stride_not_multiple_of_8(L):
+    g = _good()
+    g[3] = _t(64, 64 * 128, 124, 64, FAKE + (3 << 24))
+    _expect(L, INVALID, *g)
+
+
+def test_rejects_real_len_out_of_range(L):
+    _expect(L, INVALID, *_good(), real_len=[81])
+    _expect(L, INVALID, *_good(), real_len=[-1])
+
+
+def test_rejects_q_valid_out_of_range(L):
+    _expect(L, INVALID, *_good(), q_valid=[65])
+
+
+def test_rejects_len_mismatch(L):
+    g = _good()
+    g[2] = _t(15, 15 * 128, 128, 64, FAKE + (2 << 24))  # v_prefix shorter than k_prefix
+    _expect(L, INVALID, *g)
+    g = _good()
+    g[5] = _t(63, 63 * 128, 128, 64, FAKE + (5 << 24))  # out shorter than q
+    _expect(L, INVALID, *g)
+
+
+def test_rejects_out_aliasing_an_input(L):
+    g = _good()
+    g[5] = _t(64, 64 * 128, 128, 64, FAKE + (3 << 24) + 1024)  # inside k_suffix
+    _expect(L, INVALID, *g)
+
+
+def test_rejects_self_overlapping_out(L):
+    g = _good()
+    g[5] = _t(64, 64 * 128, 64, 64, FAKE + (5 << 24))  # stride_s < heads * head_dim
+    _expect(L, INVALID, *g)
+
+
+def test_rejects_bad_scale(L):
+    _expect(L, INVALID, *_good(), scale=float("nan"))
+    _expect(L, INVALID, *_good(), scale=-1.0)
+
+
+def test_rejects_null_pointer(L):
+    g = _good()
+    g[1] = _t(16, 16 * 128, 128, 64, None)
+    _expect(L, INVALID, *g)
+
+
+def test_wait_timeout_setter(L):
+    assert L.sk_set_wait_timeout_ms(0) == INVALID
+    assert L.sk_set_wait_timeout_ms(2000) == 0
+
+
+def test_prologue_rejects_bad_args(L):
+    q = _t(8, 8 * 256, 256, 128, FAKE)
+    k = _t(8, 8 * 128, 128, 128, FAKE + (1 << 24))
+    w = FAKE + (2 << 24)
+    tab = FAKE + (3 << 24)
+    # odd rot_dim
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 95, 0, 1e-6, 2, 1, 1, 128, None) == INVALID
+    # unsupported head_dim
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 64, 0, 1e-6, 2, 1, 1, 96, None) == UNSUPPORTED
+    # table shorter than the sequence
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 7, 96, 0, 1e-6, 2, 1, 1, 128, None) == INVALID
+    # half-split rotary width not a multiple of 16
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 72, 0, 1e-6, 2, 1, 1, 128, None) == UNSUPPORTED
+
+
+def test_python_binding_raises_on_missing_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(sk, "_lib", None)
+    monkeypatch.setattr(sk, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        sk.lib()

@@ -1,0 +1,210 @@
+"""Python binding of libsplitkv_attn (split-KV tail-padded attention for B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libsplitkv_attn.so`` behind the C ABI declared in
+``include/splitkv_attn.h``.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or a call is
+rejected, ``SplitKVError`` is raised.
+
+Entry points (same names as the C ABI):
+  attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix, real_len=None,
+                    softmax_scale=None, out=None, q_valid=None)
+  qk_rmsnorm_rope(q, k, w_q, w_k, rope_table, rot_dim=None, interleaved=False, eps=1e-6)
+  sk_device_status(device=None, clear=True), sk_set_wait_timeout_ms(ms), sk_abi_version()
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence
+
+__all__ = [
+    "SplitKVError",
+    "SkTensor",
+    "lib",
+    "attn_fwd_split_kv",
+    "qk_rmsnorm_rope",
+    "sk_device_status",
+    "sk_set_wait_timeout_ms",
+    "sk_abi_version",
+    "tensor_desc",
+    "LIB_PATH",
+    "STATUS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsplitkv_attn.so")
+
+STATUS = {0: "SK_OK", 1: "SK_ERR_INVALID_ARG", 2: "SK_ERR_UNSUPPORTED", 3: "SK_ERR_CUDA",
+          4: "SK_ERR_DEVICE_TIMEOUT"}
+
+
+class SplitKVError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = int(status)
+        self.message = message
+        super().__init__(f"{STATUS.get(self.status, self.status)}: {message}")
+
+
+class SkTensor(ctypes.Structure):
+    _fields_ = [
+        ("ptr", ctypes.c_void_p),
+        ("stride_b", ctypes.c_int64),
+        ("stride_s", ctypes.c_int64),
+        ("stride_h", ctypes.c_int64),
+        ("len_s", ctypes.c_int32),
+    ]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m varlen_flash_attention_b200.build` (nvcc, sm_100a)")
+            L = ctypes.CDLL(LIB_PATH)
+            P = ctypes.POINTER(SkTensor)
+            i32, vp = ctypes.c_int32, ctypes.c_void_p
+            L.attn_fwd_split_kv.argtypes = [P, P, P, P, P, vp, i32, i32, ctypes.c_float, P, i32, i32, vp]
+            L.attn_fwd_split_kv.restype = i32
+            L.attn_fwd_split_kv_ex.argtypes = [P, P, P, P, P, vp, i32, i32, ctypes.c_float, P, i32, i32,
+                                               vp, vp]
+            L.attn_fwd_split_kv_ex.restype = i32
+            L.qk_rmsnorm_rope.argtypes = [P, P, vp, vp, vp, i32, i32, i32, ctypes.c_float, i32, i32,
+                                          i32, i32, vp]
+            L.qk_rmsnorm_rope.restype = i32
+            L.sk_last_error.argtypes = []
+            L.sk_last_error.restype = ctypes.c_char_p
+            L.sk_device_status.argtypes = [i32, ctypes.POINTER(i32), i32]
+            L.sk_device_status.restype = i32
+            L.sk_set_wait_timeout_ms.argtypes = [i32]
+            L.sk_set_wait_timeout_ms.restype = i32
+            L.sk_abi_version.argtypes = []
+            L.sk_abi_version.restype = i32
+            _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        msg = lib().sk_last_error()
+        raise SplitKVError(status, msg.decode() if msg else "")
+
+
+def tensor_desc(t) -> SkTensor:
+    """sk_tensor_t for a 4-D BSND bf16 CUDA tensor (head_dim contiguous)."""
+    import torch
+
+    if t.dim() != 4:
+        raise ValueError("expected a 4-D [batch, seq, heads, head_dim] tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected bf16")
+    if t.numel() > 0 and not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if t.shape[3] > 1 and t.stride(3) != 1:
+        raise ValueError("head_dim must be contiguous (stride 1)")
+    return SkTensor(t.data_ptr() if t.numel() > 0 else None, t.stride(0), t.stride(1), t.stride(2),
+                    t.shape[1])
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _int32_array(vals: Optional[Sequence[int]], n: int):
+    if vals is None:
+        return None
+    vals = [int(v) for v in vals]
+    if len(vals) != n:
+        raise ValueError(f"expected {n} values, got {len(vals)}")
+    return (ctypes.c_int32 * n)(*vals)
+
+
+def attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix,
+                      real_len: Optional[Sequence[int]] = None,
+                      softmax_scale: Optional[float] = None,
+                      out=None, q_valid: Optional[Sequence[int]] = None, stream=None):
+    """Attention over cat(prefix, suffix)[:real_len[b]] without the concatenation.
+
+    q [B, Sq, Hq, D]; k/v_prefix [B, Sp, Hkv, D]; k/v_suffix [B, Ss, Hkv, D];
+    bf16 CUDA tensors (strided views allowed, head_dim contiguous).
+    real_len: host sequence of B ints (default: all Sp + Ss keys valid).
+    Returns ``out`` ([B, Sq, Hq, D] bf16, allocated if not given).
+    """
+    import torch
+
+    B, Sq, Hq, D = q.shape
+    Hkv = k_prefix.shape[2] if k_prefix.shape[1] > 0 else k_suffix.shape[2]
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=q.dtype, device=q.device)
+    if softmax_scale is None:
+        softmax_scale = D ** -0.5
+    descs = [tensor_desc(t) for t in (q, k_prefix, v_prefix, k_suffix, v_suffix, out)]
+    rl = _int32_array(real_len, B)
+    qv = _int32_array(q_valid, B)
+    L = lib()
+    args = [ctypes.byref(d) for d in descs[:5]] + [
+        ctypes.cast(rl, ctypes.c_void_p) if rl is not None else None, Hq, Hkv, float(softmax_scale),
+        ctypes.byref(descs[5]), B, D]
+    if qv is None:
+        st = L.attn_fwd_split_kv(*args, _stream_ptr(stream))
+    else:
+        st = L.attn_fwd_split_kv_ex(*args, ctypes.cast(qv, ctypes.c_void_p), _stream_ptr(stream))
+    _check(st)
+    return out
+
+
+def qk_rmsnorm_rope(q, k, w_q, w_k, rope_table, rot_dim: Optional[int] = None,
+                    interleaved: bool = False, eps: float = 1e-6, stream=None):
+    """In-place fused RMSNorm(head_dim) + RoPE on q [B,S,Hq,D] and k [B,S,Hkv,D] (bf16, CUDA).
+
+    rope_table: fp32 CUDA [rows >= S, rot_dim] holding [cos | sin]; w_q, w_k: bf16 [D].
+    """
+    import torch
+
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if rot_dim is None:
+        rot_dim = rope_table.shape[1]
+    for w in (w_q, w_k):
+        if w.dtype != torch.bfloat16 or not w.is_contiguous() or w.numel() != D:
+            raise ValueError("weights must be contiguous bf16 [head_dim]")
+    if rope_table.dtype != torch.float32 or not rope_table.is_contiguous():
+        raise ValueError("rope_table must be contiguous fp32")
+    dq, dk = tensor_desc(q), tensor_desc(k)
+    st = lib().qk_rmsnorm_rope(ctypes.byref(dq), ctypes.byref(dk), w_q.data_ptr(), w_k.data_ptr(),
+                               rope_table.data_ptr() if rope_table.numel() else None,
+                               rope_table.shape[0], int(rot_dim), int(bool(interleaved)), float(eps),
+                               Hq, Hkv, B, D, _stream_ptr(stream))
+    _check(st)
+    return q, k
+
+
+def sk_device_status(device: Optional[int] = None, clear: bool = True) -> int:
+    """Synchronise the device and return its status word (0 = no kernel gave up a wait)."""
+    import torch
+
+    if device is None:
+        device = torch.cuda.current_device()
+    v = ctypes.c_int32(0)
+    _check(lib().sk_device_status(int(device), ctypes.byref(v), int(bool(clear))))
+    return v.value
+
+
+def sk_set_wait_timeout_ms(ms: int) -> None:
+    _check(lib().sk_set_wait_timeout_ms(int(ms)))
+
+
+def sk_abi_version() -> int:
+    return int(lib().sk_abi_version())

@@ -1,0 +1,412 @@
+// C-ABI entry points of libsplitkv_attn: argument validation, per-batch
+// tensor-map encoding (extents clipped to the valid keys / query rows of each
+// batch row), launch on the caller's stream.  See include/splitkv_attn.h for
+// the contract of every function.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/splitkv_attn.h"
+#include "attn_fwd_sm100.cuh"
+#include "qk_norm_rope.cuh"
+
+namespace {
+
+constexpr int32_t kAbiVersion = 1;
+
+// ---------------------------------------------------------------- errors
+thread_local std::string g_last_error;
+
+sk_status_t fail(sk_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+sk_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(SK_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- device state
+// The status word is a module global: one per device, no allocation.
+__device__ int32_t g_device_status = 0;
+
+uint64_t g_wait_limit_ns = 2000ull * 1000ull * 1000ull;
+std::mutex g_mu;
+
+struct DeviceInfo {
+  bool checked = false;
+  bool sm100 = false;
+  int32_t* status = nullptr;
+  bool attn_attr_set[2] = {false, false};
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+
+sk_status_t device_setup(int* dev_out, DeviceInfo** info_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SK_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.sm100 = (major == 10 && minor == 0);
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_device_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    d.status = static_cast<int32_t*>(ptr);
+    d.checked = true;
+  }
+  if (!d.sm100) return fail(SK_ERR_UNSUPPORTED, "device %d is not sm_100 (B200)", dev);
+  *dev_out = dev;
+  *info_out = &d;
+  return SK_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D map over (d, head, seq) of one batch row: box = 64 d x 1 head x 128 rows,
+// 128-byte swizzle.  `rows` is the clipped sequence extent (>= 1).
+sk_status_t encode_map(CUtensorMap* m, const void* base, int64_t stride_s, int64_t stride_h,
+                       int heads, int64_t rows, int D) {
+  auto enc = get_encode_fn();
+  if (!enc) return fail(SK_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride_h) * 2u, static_cast<cuuint64_t>(stride_s) * 2u};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(skattn::kBlockM)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SK_OK;
+}
+
+// ---------------------------------------------------------------- validation helpers
+struct Span {
+  uintptr_t lo = 0, hi = 0;  // [lo, hi) bytes; empty when lo == hi
+};
+
+bool span_of(const sk_tensor_t& t, int B, int H, int D, Span* sp) {
+  if (t.len_s == 0 || B == 0) {
+    *sp = Span{};
+    return true;
+  }
+  const uintptr_t base = reinterpret_cast<uintptr_t>(t.ptr);
+  int64_t lo = 0, hi = 0;  // element offsets
+  const int64_t ext[3] = {B - 1, static_cast<int64_t>(t.len_s) - 1, H - 1};
+  const int64_t str[3] = {t.stride_b, t.stride_s, t.stride_h};
+  for (int i = 0; i < 3; ++i) {
+    const int64_t v = ext[i] * str[i];
+    if (v < 0) lo += v; else hi += v;
+  }
+  hi += D;
+  sp->lo = base + static_cast<uintptr_t>(lo * 2);
+  sp->hi = base + static_cast<uintptr_t>(hi * 2);
+  return true;
+}
+
+bool overlaps(const Span& a, const Span& b) {
+  if (a.lo == a.hi || b.lo == b.hi) return false;
+  return a.lo < b.hi && b.lo < a.hi;
+}
+
+// True when distinct (b, s, h, d) indices map to distinct elements (sufficient test:
+// sorted by stride, every stride covers the span of all smaller dimensions).
+bool no_self_overlap(const sk_tensor_t& t, int B, int H, int D) {
+  struct Dim { int64_t n, st; } dims[3] = {{B, t.stride_b}, {t.len_s, t.stride_s}, {H, t.stride_h}};
+  std::sort(dims, dims + 3, [](const Dim& a, const Dim& b) { return a.st < b.st; });
+  int64_t span = D;  // d is contiguous
+  for (auto& d : dims) {
+    if (d.n <= 1) continue;
+    if (d.st < span) return false;
+    span = d.st * (d.n - 1) + span;
+  }
+  return true;
+}
+
+sk_status_t check_tensor(const char* name, const sk_tensor_t* t, int B, int H, int D) {
+  if (!t) return fail(SK_ERR_INVALID_ARG, "%s: NULL descriptor", name);
+  if (t->len_s < 0) return fail(SK_ERR_INVALID_ARG, "%s: negative len_s", name);
+  if (t->len_s == 0 || B == 0) return SK_OK;
+  if (!t->ptr) return fail(SK_ERR_INVALID_ARG, "%s: NULL ptr with len_s > 0", name);
+  if (reinterpret_cast<uintptr_t>(t->ptr) % 16 != 0)
+    return fail(SK_ERR_INVALID_ARG, "%s: ptr not 16-byte aligned", name);
+  const int64_t st[3] = {t->stride_b, t->stride_s, t->stride_h};
+  const char* nm[3] = {"stride_b", "stride_s", "stride_h"};
+  for (int i = 0; i < 3; ++i) {
+    if (st[i] % 8 != 0) return fail(SK_ERR_INVALID_ARG, "%s: %s=%lld not a multiple of 8 elements", name, nm[i], (long long)st[i]);
+    if (st[i] < 0) return fail(SK_ERR_INVALID_ARG, "%s: %s negative", name, nm[i]);
+    if (st[i] * 2 >= (int64_t(1) << 40)) return fail(SK_ERR_INVALID_ARG, "%s: %s too large", name, nm[i]);
+  }
+  if (H > 1 && t->stride_h == 0) return fail(SK_ERR_INVALID_ARG, "%s: stride_h is 0", name);
+  if (t->len_s > 1 && t->stride_s == 0) return fail(SK_ERR_INVALID_ARG, "%s: stride_s is 0", name);
+  return SK_OK;
+}
+
+template <int D>
+sk_status_t launch_attn(const skattn::AttnParams& prm, int n_qtiles, int H, int nb, cudaStream_t stream,
+                        DeviceInfo* dev) {
+  using L = skattn::SmemLayout<D>;
+  const int slot = (D == 64) ? 0 : 1;
+  if (!dev->attn_attr_set[slot]) {
+    cudaError_t e = cudaFuncSetAttribute(skattn::attn_fwd_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    dev->attn_attr_set[slot] = true;
+  }
+  dim3 grid(n_qtiles, H, nb);
+  skattn::attn_fwd_kernel<D><<<grid, skattn::kThreads, L::kAlloc, stream>>>(prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  return SK_OK;
+}
+
+sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tensor_t* vp,
+                      const sk_tensor_t* ks, const sk_tensor_t* vs, const int32_t* real_len,
+                      int32_t Hq, int32_t Hkv, float scale, const sk_tensor_t* out, int32_t B,
+                      int32_t D, const int32_t* q_valid_in, void* stream_v) {
+  if (B < 0) return fail(SK_ERR_INVALID_ARG, "batch < 0");
+  if (Hq <= 0 || Hkv <= 0) return fail(SK_ERR_INVALID_ARG, "head counts must be positive");
+  if (Hq % Hkv != 0) return fail(SK_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
+  if (Hq > 65535) return fail(SK_ERR_UNSUPPORTED, "num_q_heads > 65535");
+  if (D != 64 && D != 128) return fail(SK_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", D);
+  if (!(std::isfinite(scale) && scale >= 0.f)) return fail(SK_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  sk_status_t st;
+  if ((st = check_tensor("q", q, B, Hq, D)) != SK_OK) return st;
+  if ((st = check_tensor("k_prefix", kp, B, Hkv, D)) != SK_OK) return st;
+  if ((st = check_tensor("v_prefix", vp, B, Hkv, D)) != SK_OK) return st;
+  if ((st = check_tensor("k_suffix", ks, B, Hkv, D)) != SK_OK) return st;
+  if ((st = check_tensor("v_suffix", vs, B, Hkv, D)) != SK_OK) return st;
+  if ((st = check_tensor("out", out, B, Hq, D)) != SK_OK) return st;
+  const int32_t Sq = q->len_s;
+  if (out->len_s != Sq) return fail(SK_ERR_INVALID_ARG, "out.len_s (%d) != q.len_s (%d)", out->len_s, Sq);
+  if (kp->len_s != vp->len_s) return fail(SK_ERR_INVALID_ARG, "k_prefix.len_s != v_prefix.len_s");
+  if (ks->len_s != vs->len_s) return fail(SK_ERR_INVALID_ARG, "k_suffix.len_s != v_suffix.len_s");
+  const int64_t Sp = kp->len_s, Ss = ks->len_s, Skv = Sp + Ss;
+  if (Skv > INT32_MAX) return fail(SK_ERR_INVALID_ARG, "Sp + Ss too large");
+  if (!no_self_overlap(*out, B, Hq, D)) return fail(SK_ERR_INVALID_ARG, "out overlaps itself");
+  if (B == 0 || Sq == 0) return SK_OK;
+  Span so, si;
+  span_of(*out, B, Hq, D, &so);
+  const struct { const char* n; const sk_tensor_t* t; int H; } ins[5] = {
+      {"q", q, Hq}, {"k_prefix", kp, Hkv}, {"v_prefix", vp, Hkv}, {"k_suffix", ks, Hkv}, {"v_suffix", vs, Hkv}};
+  for (auto& in : ins) {
+    span_of(*in.t, B, in.H, D, &si);
+    if (overlaps(so, si)) return fail(SK_ERR_INVALID_ARG, "out overlaps %s", in.n);
+  }
+  for (int b = 0; b < B; ++b) {
+    const int64_t n = real_len ? real_len[b] : Skv;
+    if (n < 0 || n > Skv) return fail(SK_ERR_INVALID_ARG, "real_len[%d]=%lld outside [0, %lld]", b, (long long)n, (long long)Skv);
+    if (q_valid_in && (q_valid_in[b] < 0 || q_valid_in[b] > Sq))
+      return fail(SK_ERR_INVALID_ARG, "q_valid[%d]=%d outside [0, %d]", b, q_valid_in[b], Sq);
+  }
+
+  int dev = 0;
+  DeviceInfo* info = nullptr;
+  if ((st = device_setup(&dev, &info)) != SK_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+
+  const int n_qtiles = (Sq + skattn::kBlockM - 1) / skattn::kBlockM;
+  for (int b0 = 0; b0 < B; b0 += skattn::kMaxBatch) {
+    const int nb = std::min(skattn::kMaxBatch, B - b0);
+    skattn::AttnParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    for (int i = 0; i < nb; ++i) {
+      const int b = b0 + i;
+      const int64_t n = real_len ? real_len[b] : Skv;
+      const int64_t npre = std::min<int64_t>(Sp, n);
+      const int64_t nsuf = std::max<int64_t>(0, n - Sp);
+      // joint self-attention (Sq == Skv): the tail pad covers the query stream too
+      const int64_t qv = q_valid_in ? q_valid_in[b] : (Sq == Skv ? n : Sq);
+      prm.q_valid[i] = static_cast<int32_t>(qv);
+      prm.n_prefix[i] = static_cast<int32_t>(npre);
+      prm.n_suffix[i] = static_cast<int32_t>(nsuf);
+      auto bptr = [&](const sk_tensor_t* t) {
+        return static_cast<const void*>(static_cast<const uint16_t*>(t->ptr) + static_cast<int64_t>(b) * t->stride_b);
+      };
+      if (qv > 0 && n > 0)
+        if ((st = encode_map(&prm.tm_q[i], bptr(q), q->stride_s, q->stride_h, Hq, qv, D)) != SK_OK) return st;
+      if (npre > 0) {
+        if ((st = encode_map(&prm.tm_kp[i], bptr(kp), kp->stride_s, kp->stride_h, Hkv, npre, D)) != SK_OK) return st;
+        if ((st = encode_map(&prm.tm_vp[i], bptr(vp), vp->stride_s, vp->stride_h, Hkv, npre, D)) != SK_OK) return st;
+      }
+      if (nsuf > 0) {
+        if ((st = encode_map(&prm.tm_ks[i], bptr(ks), ks->stride_s, ks->stride_h, Hkv, nsuf, D)) != SK_OK) return st;
+        if ((st = encode_map(&prm.tm_vs[i], bptr(vs), vs->stride_s, vs->stride_h, Hkv, nsuf, D)) != SK_OK) return st;
+      }
+    }
+    prm.out = static_cast<uint16_t*>(out->ptr) + static_cast<int64_t>(b0) * out->stride_b;
+    prm.out_sb = out->stride_b;
+    prm.out_ss = out->stride_s;
+    prm.out_sh = out->stride_h;
+    prm.Sq = Sq;
+    prm.group = Hq / Hkv;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.status = info->status;
+    prm.wait_limit_ns = g_wait_limit_ns;
+    st = (D == 64) ? launch_attn<64>(prm, n_qtiles, Hq, nb, stream, info)
+                   : launch_attn<128>(prm, n_qtiles, Hq, nb, stream, info);
+    if (st != SK_OK) return st;
+  }
+  return SK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sk_status_t attn_fwd_split_kv(const sk_tensor_t* q, const sk_tensor_t* k_prefix, const sk_tensor_t* v_prefix,
+                              const sk_tensor_t* k_suffix, const sk_tensor_t* v_suffix, const int32_t* real_len,
+                              int32_t num_q_heads, int32_t num_kv_heads, float softmax_scale,
+                              const sk_tensor_t* out, int32_t batch, int32_t head_dim, void* stream) {
+  try {
+    return attn_impl(q, k_prefix, v_prefix, k_suffix, v_suffix, real_len, num_q_heads, num_kv_heads,
+                     softmax_scale, out, batch, head_dim, nullptr, stream);
+  } catch (...) {
+    return fail(SK_ERR_INVALID_ARG, "internal exception");
+  }
+}
+
+sk_status_t attn_fwd_split_kv_ex(const sk_tensor_t* q, const sk_tensor_t* k_prefix,
+                                 const sk_tensor_t* v_prefix, const sk_tensor_t* k_suffix,
+                                 const sk_tensor_t* v_suffix, const int32_t* real_len,
+                                 int32_t num_q_heads, int32_t num_kv_heads, float softmax_scale,
+                                 const sk_tensor_t* out, int32_t batch, int32_t head_dim,
+                                 const int32_t* q_valid, void* stream) {
+  try {
+    return attn_impl(q, k_prefix, v_prefix, k_suffix, v_suffix, real_len, num_q_heads, num_kv_heads,
+                     softmax_scale, out, batch, head_dim, q_valid, stream);
+  } catch (...) {
+    return fail(SK_ERR_INVALID_ARG, "internal exception");
+  }
+}
+
+sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, const void* w_q, const void* w_k,
+                            const float* rope_table, int32_t table_rows, int32_t rot_dim,
+                            int32_t interleaved, float eps, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t batch, int32_t head_dim, void* stream) {
+  try {
+    if (batch < 0) return fail(SK_ERR_INVALID_ARG, "batch < 0");
+    if (num_q_heads <= 0 || num_kv_heads <= 0) return fail(SK_ERR_INVALID_ARG, "head counts must be positive");
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+      return fail(SK_ERR_UNSUPPORTED, "head_dim %d not in {64, 128, 256}", head_dim);
+    if (rot_dim < 0 || rot_dim > head_dim || (rot_dim & 1)) return fail(SK_ERR_INVALID_ARG, "rot_dim must be even and in [0, head_dim]");
+    if (!(std::isfinite(eps) && eps >= 0.f)) return fail(SK_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    sk_status_t st;
+    if ((st = check_tensor("q", q, batch, num_q_heads, head_dim)) != SK_OK) return st;
+    if ((st = check_tensor("k", k, batch, num_kv_heads, head_dim)) != SK_OK) return st;
+    if (q->len_s != k->len_s) return fail(SK_ERR_INVALID_ARG, "q.len_s != k.len_s");
+    const int32_t S = q->len_s;
+    if (batch == 0 || S == 0) return SK_OK;
+    if (!no_self_overlap(*q, batch, num_q_heads, head_dim) || !no_self_overlap(*k, batch, num_kv_heads, head_dim))
+      return fail(SK_ERR_INVALID_ARG, "q or k overlaps itself");
+    Span sq, sk;
+    span_of(*q, batch, num_q_heads, head_dim, &sq);
+    span_of(*k, batch, num_kv_heads, head_dim, &sk);
+    if (overlaps(sq, sk)) {
+      // allowed only when they are disjoint head ranges of one fused buffer; require distinct elements
+      // by checking that q's heads and k's heads never share an address: same strides, k after q's heads.
+      const bool fused = q->stride_b == k->stride_b && q->stride_s == k->stride_s && q->stride_h == k->stride_h &&
+                         static_cast<const uint16_t*>(k->ptr) >= static_cast<const uint16_t*>(q->ptr) + num_q_heads * q->stride_h;
+      if (!fused) return fail(SK_ERR_INVALID_ARG, "q and k overlap");
+    }
+    if (!w_q || !w_k || (rot_dim > 0 && !rope_table)) return fail(SK_ERR_INVALID_ARG, "NULL weight or table");
+    if (reinterpret_cast<uintptr_t>(w_q) % 16 || reinterpret_cast<uintptr_t>(w_k) % 16 ||
+        reinterpret_cast<uintptr_t>(rope_table) % 16)
+      return fail(SK_ERR_INVALID_ARG, "weights and table must be 16-byte aligned");
+    if (rot_dim > 0 && table_rows < S) return fail(SK_ERR_INVALID_ARG, "table_rows < seq len");
+    if (interleaved && rot_dim % 8 != 0)
+      return fail(SK_ERR_UNSUPPORTED, "interleaved rot_dim must be a multiple of 8");
+    if (!interleaved && rot_dim % 16 != 0)
+      return fail(SK_ERR_UNSUPPORTED, "half-split rot_dim must be a multiple of 16");
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    if ((st = device_setup(&dev, &info)) != SK_OK) return st;
+    skqkn::NormRopeParams prm;
+    prm.q = static_cast<uint16_t*>(q->ptr);
+    prm.k = static_cast<uint16_t*>(k->ptr);
+    prm.q_sb = q->stride_b; prm.q_ss = q->stride_s; prm.q_sh = q->stride_h;
+    prm.k_sb = k->stride_b; prm.k_ss = k->stride_s; prm.k_sh = k->stride_h;
+    prm.w_q = static_cast<const uint16_t*>(w_q);
+    prm.w_k = static_cast<const uint16_t*>(w_k);
+    prm.table = rope_table;
+    prm.rot_dim = rot_dim;
+    prm.interleaved = interleaved != 0;
+    prm.eps = eps;
+    prm.S = S;
+    prm.Hq = num_q_heads;
+    prm.Hkv = num_kv_heads;
+    prm.B = batch;
+    cudaError_t e = skqkn::launch(prm, head_dim, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "qk_rmsnorm_rope launch");
+    return SK_OK;
+  } catch (...) {
+    return fail(SK_ERR_INVALID_ARG, "internal exception");
+  }
+}
+
+const char* sk_last_error(void) { return g_last_error.c_str(); }
+
+sk_status_t sk_device_status(int32_t device, int32_t* status_out, int32_t clear) {
+  if (!status_out) return fail(SK_ERR_INVALID_ARG, "status_out is NULL");
+  int prev = 0;
+  cudaError_t e = cudaGetDevice(&prev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (device != prev && (e = cudaSetDevice(device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  sk_status_t st = SK_OK;
+  int32_t v = 0;
+  e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof v);
+  if (e == cudaSuccess && clear) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero);
+  }
+  if (e != cudaSuccess) st = cuda_fail(e, "reading device status");
+  *status_out = v;
+  if (device != prev) cudaSetDevice(prev);
+  return st;
+}
+
+sk_status_t sk_set_wait_timeout_ms(int32_t ms) {
+  if (ms < 1 || ms > 60000) return fail(SK_ERR_INVALID_ARG, "timeout must be in [1, 60000] ms");
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_wait_limit_ns = static_cast<uint64_t>(ms) * 1000000ull;
+  return SK_OK;
+}
+
+int32_t sk_abi_version(void) { return kAbiVersion; }
+
+}  // extern "C"
