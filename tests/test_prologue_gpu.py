@@ -1,8 +1,9 @@
 """Parity of the fused Q/K RMSNorm + RoPE prologue kernel with the fp64 oracle.
 
-Bar: every output element within 1 bf16 ulp of the oracle (the kernel's fp32
-rsqrt and products may land on the other side of a bf16 rounding boundary),
-and at least 99% of elements bit-identical.
+Bar: every output element within 1 bf16 ulp of the oracle and at least
+99.99% bit-identical.  The kernel computes in fp64 with the oracle's rounding
+points, so in practice every element is identical; the ulp allowance covers a
+sum-of-squares reduction order that differs from the oracle's sequential one.
 """
 import numpy as np
 import pytest
@@ -40,7 +41,7 @@ def _ulp_check(got_bits, ref_bits):
     b = np.where(b & 0x8000, -(b & 0x7FFF), b)
     d = np.abs(a - b)
     assert d.max() <= 1, d.max()
-    assert (d == 0).mean() >= 0.99, (d == 0).mean()
+    assert (d == 0).mean() >= 0.9999, (d == 0).mean()
 
 
 @pytest.mark.parametrize("D,rot,inter", [(128, 96, False), (128, 128, False), (128, 96, True),
@@ -54,10 +55,11 @@ def test_prologue_matches_oracle(sk, D, rot, inter):
     wq = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
     wk = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
     tab = _table(S + 5, rot) if rot else torch.zeros(S, 0)
+    eps = float(np.float32(1e-6))  # the C ABI takes eps as fp32
     ref_q = oracle.qk_rmsnorm_rope(q, wq, tab.numpy() if rot else np.zeros((S, 0), np.float32),
-                                   rot_dim=rot, interleaved=inter, eps=1e-6)
+                                   rot_dim=rot, interleaved=inter, eps=eps)
     ref_k = oracle.qk_rmsnorm_rope(k, wk, tab.numpy() if rot else np.zeros((S, 0), np.float32),
-                                   rot_dim=rot, interleaved=inter, eps=1e-6)
+                                   rot_dim=rot, interleaved=inter, eps=eps)
     qd, kd = q.cuda(), k.cuda()
     tabd = tab.cuda() if rot else torch.zeros(S, 8, device="cuda")
     sk.qk_rmsnorm_rope(qd, kd, wq.cuda(), wk.cuda(), tabd, rot_dim=rot, interleaved=inter, eps=1e-6)
@@ -78,7 +80,8 @@ def test_prologue_in_place_on_fused_qkv_view(sk):
     torch.cuda.synchronize()
     got = d.cpu()
     assert torch.equal(got[:, :, Hq + Hkv:], qkv[:, :, Hq + Hkv:])  # v untouched
-    ref_q = oracle.qk_rmsnorm_rope(qkv[:, :, :Hq].contiguous(), wq, tab.numpy(), eps=1e-5)
-    ref_k = oracle.qk_rmsnorm_rope(qkv[:, :, Hq:Hq + Hkv].contiguous(), wk, tab.numpy(), eps=1e-5)
+    eps = float(np.float32(1e-5))
+    ref_q = oracle.qk_rmsnorm_rope(qkv[:, :, :Hq].contiguous(), wq, tab.numpy(), eps=eps)
+    ref_k = oracle.qk_rmsnorm_rope(qkv[:, :, Hq:Hq + Hkv].contiguous(), wk, tab.numpy(), eps=eps)
     _ulp_check(got[:, :, :Hq].contiguous().view(torch.int16).numpy().view(np.uint16), ref_q)
     _ulp_check(got[:, :, Hq:Hq + Hkv].contiguous().view(torch.int16).numpy().view(np.uint16), ref_k)

@@ -7,8 +7,11 @@
 // xor-shuffles inside the row's lane group; in half-split (NeoX) mode the
 // rotation partner (d + rot_dim/2) lives rot_dim/16 lanes away and is fetched
 // with one shuffle of the already bf16-rounded normalised values.
-// Rounding follows the unfused path: RMSNorm output rounded to bf16, rotation
-// in fp32, result rounded to bf16 (nearest even).
+// Rounding follows the unfused path: RMSNorm output rounded to bf16, rotation,
+// result rounded to bf16 (nearest even).  The arithmetic is fp64: the kernel is
+// bound by HBM, and in fp64 every product of a bf16 value with an fp32 table
+// entry is exact, so the one rounding before each bf16 store is the only one
+// that matters (fp32 is not enough when the rotation cancels).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -31,18 +34,27 @@ struct NormRopeParams {
   int S, Hq, Hkv, B;
 };
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
+// Nearest-even bf16 of a double, rounded once: through fp32 (nearest), then to
+// bf16, correcting the one case where the fp32 step lands exactly on a bf16
+// midpoint that the double was not on.
+__device__ __forceinline__ uint32_t bf16_bits_rn(double x) {
+  const float f = __double2float_rn(x);
+  const uint32_t u = __float_as_uint(f);
+  if ((u & 0x7F800000u) == 0x7F800000u) return (u & 0x7FFFFFFFu) > 0x7F800000u ? 0x7FC0u : (u >> 16);
+  uint32_t up = u >> 16;
+  const uint32_t low = u & 0xFFFFu;
+  if (low > 0x8000u) {
+    up += 1;
+  } else if (low == 0x8000u) {
+    const double fd = static_cast<double>(f);
+    if (fd == x) up += (up & 1u);
+    else if (fabs(x) > fabs(fd)) up += 1;
+  }
+  return up;
 }
 
-__device__ __forceinline__ float round_bf16(float x) {
-  uint32_t r = pack2(x, 0.f);
-  return bf16lo(r);
+__device__ __forceinline__ double bf16_to_f64(uint32_t bits16) {
+  return static_cast<double>(__uint_as_float(bits16 << 16));
 }
 
 template <int D>
@@ -77,29 +89,33 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const NormRopeParams 
   }
   const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
   const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-  float x[8], wf[8];
+  double x[8], wf[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    x[2 * i] = bf16lo(xw[i]);
-    x[2 * i + 1] = bf16hi(xw[i]);
-    wf[2 * i] = bf16lo(ww[i]);
-    wf[2 * i + 1] = bf16hi(ww[i]);
+    x[2 * i] = bf16_to_f64(xw[i] & 0xFFFFu);
+    x[2 * i + 1] = bf16_to_f64(xw[i] >> 16);
+    wf[2 * i] = bf16_to_f64(ww[i] & 0xFFFFu);
+    wf[2 * i + 1] = bf16_to_f64(ww[i] >> 16);
   }
-  float ss = 0.f;
+  double ss = 0.0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+  for (int i = 0; i < 8; ++i) ss += x[i] * x[i];
 #pragma unroll
   for (int o = TPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float r = rsqrtf(ss * (1.0f / D) + p.eps);
-  float y[8];
+  const double r = 1.0 / sqrt(ss / static_cast<double>(D) + static_cast<double>(p.eps));
+  uint32_t yb[8];
+  double y[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) y[i] = round_bf16(x[i] * r * wf[i]);
+  for (int i = 0; i < 8; ++i) {
+    yb[i] = bf16_bits_rn(x[i] * r * wf[i]);
+    y[i] = bf16_to_f64(yb[i]);
+  }
 
   const int d0 = sub * 8;
   const int rot = p.rot_dim;
-  float z[8];
+  uint32_t zb[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) z[i] = y[i];
+  for (int i = 0; i < 8; ++i) zb[i] = yb[i];
 
   if (p.interleaved) {
     if (valid && d0 < rot) {
@@ -110,9 +126,9 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const NormRopeParams 
       const float sn[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float a = y[2 * e], c = y[2 * e + 1];
-        z[2 * e] = fmaf(a, cs[e], -(c * sn[e]));
-        z[2 * e + 1] = fmaf(c, cs[e], a * sn[e]);
+        const double a = y[2 * e], c = y[2 * e + 1];
+        zb[2 * e] = bf16_bits_rn(a * static_cast<double>(cs[e]) - c * static_cast<double>(sn[e]));
+        zb[2 * e + 1] = bf16_bits_rn(c * static_cast<double>(cs[e]) + a * static_cast<double>(sn[e]));
       }
     }
   } else {
@@ -124,13 +140,13 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const NormRopeParams 
     const int src = (lane & ~(TPR - 1)) + psub;
     uint32_t yp[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) yp[i] = __shfl_sync(0xffffffffu, pack2(y[2 * i], y[2 * i + 1]), src);
+    for (int i = 0; i < 4; ++i) yp[i] = __shfl_sync(0xffffffffu, yb[2 * i] | (yb[2 * i + 1] << 16), src);
     if (valid && (first || second)) {
-      float ypart[8];
+      double ypart[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        ypart[2 * i] = bf16lo(yp[i]);
-        ypart[2 * i + 1] = bf16hi(yp[i]);
+        ypart[2 * i] = bf16_to_f64(yp[i] & 0xFFFFu);
+        ypart[2 * i + 1] = bf16_to_f64(yp[i] >> 16);
       }
       const int i0 = first ? d0 : d0 - half;
       const float* crow = p.table + static_cast<int64_t>(s) * rot;
@@ -142,19 +158,21 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const NormRopeParams 
       const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
       if (first) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) z[e] = fmaf(y[e], cs[e], -(ypart[e] * sn[e]));
+        for (int e = 0; e < 8; ++e)
+          zb[e] = bf16_bits_rn(y[e] * static_cast<double>(cs[e]) - ypart[e] * static_cast<double>(sn[e]));
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) z[e] = fmaf(y[e], cs[e], ypart[e] * sn[e]);
+        for (int e = 0; e < 8; ++e)
+          zb[e] = bf16_bits_rn(y[e] * static_cast<double>(cs[e]) + ypart[e] * static_cast<double>(sn[e]));
       }
     }
   }
   if (valid) {
     uint4 o;
-    o.x = pack2(z[0], z[1]);
-    o.y = pack2(z[2], z[3]);
-    o.z = pack2(z[4], z[5]);
-    o.w = pack2(z[6], z[7]);
+    o.x = zb[0] | (zb[1] << 16);
+    o.y = zb[2] | (zb[3] << 16);
+    o.z = zb[4] | (zb[5] << 16);
+    o.w = zb[6] | (zb[7] << 16);
     *reinterpret_cast<uint4*>(ptr) = o;
   }
 }
