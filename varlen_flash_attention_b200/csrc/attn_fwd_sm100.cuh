@@ -1,24 +1,30 @@
 // Split-KV tail-padded attention forward for sm_100a.
 //
-// One CTA computes one 128-row query tile of one (batch row, query head):
+// One CTA computes two 128-row query tiles (A and B, 256 consecutive rows) of
+// one (batch row, query head):
 //   O = softmax(scale * Q K*^T) V*,  K*/V* = cat(prefix, suffix)[0:real_len]
 // ("sglang PR 26973", forward_with_replicated_kv_prefix; "sglang PR 30107",
 // tail_attn_meta / tail-pad layout invariant).  The concatenation is never
 // built: the KV tile loop first walks the prefix tensor map, then the suffix
 // tensor map.  Each map's sequence extent is clipped on the host to the valid
-// keys of this batch row, so TMA never fetches a pad byte (out-of-range rows
-// arrive as zeros) and tiles past real_len are never issued; the one partial
-// tile of each source is masked column-wise in the softmax.
+// keys of this batch row, so TMA never fetches a pad byte (rows past the
+// extent arrive as zeros) and tiles past real_len are never issued; the one
+// partial tile of each source is masked column-wise in the softmax.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t of the tile (TMEM lane t);
-//              online softmax in fp32 (exp2 with scale*log2(e) folded in),
-//              P written back to TMEM as bf16, O rescaled in TMEM, epilogue.
-//   warp 4     TMA producer: Q once, then K/V tiles into a 2-stage ring.
-//   warp 5     TMEM allocator + single-thread tcgen05.mma issuer:
-//              S_j = Q K_j^T (SS, both K-major) into one of two S buffers,
-//              O += P_{j-1} V_{j-1} (A = P from TMEM, B = V MN-major).
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256, 256+D).
+// Warp roles (320 threads):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread t of a
+//              warpgroup owns query row t of its tile (TMEM lane t).  Online
+//              softmax in fp32 with exp2 (scale*log2 e folded in); the running
+//              max is only raised when a tile's max exceeds it by more than
+//              kRescaleLog2 (then O and l are rescaled), so most tiles skip the
+//              O round trip through registers.  P goes back to TMEM as bf16,
+//              over the first 64 columns of the tile's S buffer.
+//   warp 8     TMA producer: both Q tiles once, then K and V tiles into rings.
+//   warp 9     TMEM allocator + single-thread tcgen05.mma issuer.  Two
+//              independent chains, S_X(j) -> softmax_X(j) -> PV_X(j) ->
+//              S_X(j+1) for X in {A, B}, interleave on the tensor pipe so one
+//              tile's softmax overlaps the other tile's MMAs.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
 // Every wait is bounded (globaltimer); on expiry the CTA raises a device
 // status word, drains its own copies, frees TMEM and exits.
 #pragma once
@@ -32,13 +38,17 @@
 
 namespace skattn {
 
-constexpr int kBlockM = 128;    // query rows per tile
-constexpr int kBlockN = 128;    // keys per KV tile
-constexpr int kMaxBatch = 8;    // batch rows per launch (tensor maps live in parameter space)
-constexpr int kThreads = 192;
-constexpr int kStages = 2;      // K/V smem ring depth
+constexpr int kBlockM = 128;     // query rows per tile
+constexpr int kTilesPerCta = 2;  // query tiles per CTA
+constexpr int kRowsPerCta = kBlockM * kTilesPerCta;
+constexpr int kBlockN = 128;     // keys per KV tile
+constexpr int kMaxBatch = 8;     // batch rows per launch (tensor maps live in parameter space)
+constexpr int kThreads = 320;
+constexpr int kKStages = 2;      // K smem ring depth
+constexpr int kVStages = 2;      // V smem ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr int32_t kStatusTimeout = 4;
+constexpr float kRescaleLog2 = 8.0f;  // keep a stale max while the new one is within 2^8
 
 struct alignas(64) AttnParams {
   CUtensorMap tm_q[kMaxBatch];
@@ -61,22 +71,23 @@ struct alignas(64) AttnParams {
 template <int D>
 struct SmemLayout {
   static_assert(D == 64 || D == 128, "head_dim");
-  static constexpr uint32_t kSub = kBlockM * 128;          // one 64-column (128 B) swizzled sub-tile
-  static constexpr uint32_t kQBytes = kBlockM * D * 2;
-  static constexpr uint32_t kKVBytes = kBlockN * D * 2;
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kQBytes;
-  static constexpr uint32_t kV = kK + kStages * kKVBytes;
-  static constexpr uint32_t kBar = kV + kStages * kKVBytes;
+  static constexpr uint32_t kSub = kBlockM * 128;  // one 64-column (128 B) swizzled sub-tile
+  static constexpr uint32_t kQTile = kBlockM * D * 2;
+  static constexpr uint32_t kKVTile = kBlockN * D * 2;
+  static constexpr uint32_t kQ = 0;                                  // + tile * kQTile
+  static constexpr uint32_t kK = kQ + kTilesPerCta * kQTile;         // + stage * kKVTile
+  static constexpr uint32_t kV = kK + kKStages * kKVTile;            // + stage * kKVTile
+  static constexpr uint32_t kBar = kV + kVStages * kKVTile;
   // barrier indices
   static constexpr int bQFull = 0;
-  static constexpr int bKFull = 1;                   // + stage
-  static constexpr int bVFull = bKFull + kStages;    // + stage
-  static constexpr int bKVEmpty = bVFull + kStages;  // + stage
-  static constexpr int bSFull = bKVEmpty + kStages;  // + buffer (2)
-  static constexpr int bPFull = bSFull + 2;          // + buffer (2)
-  static constexpr int bOReady = bPFull + 2;
-  static constexpr int bMmaDone = bOReady + 1;
+  static constexpr int bKFull = 1;                     // + stage
+  static constexpr int bKEmpty = bKFull + kKStages;    // + stage
+  static constexpr int bVFull = bKEmpty + kKStages;    // + stage
+  static constexpr int bVEmpty = bVFull + kVStages;    // + stage
+  static constexpr int bSFull = bVEmpty + kVStages;    // + tile
+  static constexpr int bPFull = bSFull + kTilesPerCta; // + tile
+  static constexpr int bOReady = bPFull + kTilesPerCta;// + tile
+  static constexpr int bMmaDone = bOReady + kTilesPerCta;
   static constexpr int kNumBars = bMmaDone + 1;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
   static constexpr uint32_t kEnd = kMisc + 16;
@@ -121,6 +132,34 @@ __device__ __forceinline__ void store_zero_rows(uint16_t* base, int64_t ss, int 
   }
 }
 
+// Valid keys in KV tile j (prefix tiles first, then suffix tiles).
+__device__ __forceinline__ int tile_valid(int j, int tP, int nkp, int nks) {
+  return (j < tP) ? min(kBlockN, nkp - j * kBlockN) : min(kBlockN, nks - (j - tP) * kBlockN);
+}
+
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t sQ, uint32_t sK) {
+  using L = SmemLayout<D>;
+  constexpr uint32_t idS = skptx::idesc_bf16_f32(kBlockM, kBlockN, false);
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t off = (k / 4) * L::kSub + (k % 4) * 32;
+    skptx::mma_ss(d_tmem, skptx::sdesc_sw128(sQ + off, 16, 1024), skptx::sdesc_sw128(sK + off, 16, 1024),
+                  idS, k > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t sV, bool accumulate) {
+  using L = SmemLayout<D>;
+  constexpr uint32_t idO = skptx::idesc_bf16_f32(kBlockM, D, true);
+#pragma unroll
+  for (int k = 0; k < kBlockN / 16; ++k) {
+    skptx::mma_ts(o_tmem, p_tmem + k * 8, skptx::sdesc_sw128(sV + k * 2048, L::kSub, 1024), idO,
+                  (accumulate || k > 0) ? 1u : 0u);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using L = SmemLayout<D>;
@@ -131,10 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  const int q_tile = blockIdx.x;
   const int hq = blockIdx.y;
   const int bl = blockIdx.z;
-  const int row0 = q_tile * kBlockM;
+  const int row0 = blockIdx.x * kRowsPerCta;
   const int qv = p.q_valid[bl];
   const int nkp = p.n_prefix[bl];
   const int nks = p.n_suffix[bl];
@@ -144,8 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   uint16_t* out_bh = p.out + static_cast<int64_t>(bl) * p.out_sb + static_cast<int64_t>(hq) * p.out_sh;
 
   if (row0 >= qv || n_tiles == 0) {
-    // The whole tile is pad rows, or this batch row has no valid key: exact zeros.
-    const int r_end = min(row0 + kBlockM, p.Sq);
+    // Every row of this CTA is pad, or this batch row has no valid key: exact zeros.
+    const int r_end = min(row0 + kRowsPerCta, p.Sq);
     store_zero_rows(out_bh, p.out_ss, row0, r_end, D, threadIdx.x, kThreads);
     return;
   }
@@ -156,21 +194,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     skptx::mbar_init(bar(L::bQFull), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       skptx::mbar_init(bar(L::bKFull + s), 1);
+      skptx::mbar_init(bar(L::bKEmpty + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       skptx::mbar_init(bar(L::bVFull + s), 1);
-      skptx::mbar_init(bar(L::bKVEmpty + s), 1);
+      skptx::mbar_init(bar(L::bVEmpty + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      skptx::mbar_init(bar(L::bSFull + b), 1);
-      skptx::mbar_init(bar(L::bPFull + b), kBlockM);
+    for (int x = 0; x < kTilesPerCta; ++x) {
+      skptx::mbar_init(bar(L::bSFull + x), 1);
+      skptx::mbar_init(bar(L::bPFull + x), kBlockM);
+      skptx::mbar_init(bar(L::bOReady + x), 1);
     }
-    skptx::mbar_init(bar(L::bOReady), 1);
     skptx::mbar_init(bar(L::bMmaDone), 1);
     *abort_flag = 0;
     skptx::fence_mbarrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     skptx::tmem_alloc(skptx::smem_addr(tmem_slot), kTmemCols);
     skptx::tmem_relinquish();
   }
@@ -180,108 +221,116 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int hkv = hq / p.group;
       skptx::prefetch_tmap(&p.tm_q[bl]);
       if (tP > 0) { skptx::prefetch_tmap(&p.tm_kp[bl]); skptx::prefetch_tmap(&p.tm_vp[bl]); }
       if (tS > 0) { skptx::prefetch_tmap(&p.tm_ks[bl]); skptx::prefetch_tmap(&p.tm_vs[bl]); }
-      skptx::mbar_arrive_expect_tx(bar(L::bQFull), L::kQBytes);
+      skptx::mbar_arrive_expect_tx(bar(L::bQFull), kTilesPerCta * L::kQTile);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        skptx::tma_load_3d(sbase + L::kQ + c * L::kSub, &p.tm_q[bl], bar(L::bQFull), c * 64, hq, row0);
-      int j = 0;
-      for (; j < n_tiles; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages && !W.wait(bar(L::bKVEmpty + s), ((j / kStages) - 1) & 1)) break;
+      for (int x = 0; x < kTilesPerCta; ++x)
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          skptx::tma_load_3d(sbase + L::kQ + x * L::kQTile + c * L::kSub, &p.tm_q[bl], bar(L::bQFull),
+                             c * 64, hq, row0 + x * kBlockM);
+      // K(j) is issued one tile ahead of V(j): S needs K first, PV needs V later.
+      int jk = 0, jv = 0;
+      bool ok = true;
+      while (ok && (jk < n_tiles || jv < n_tiles)) {
+        const bool do_k = jk < n_tiles && jk <= jv + 1;
+        const int j = do_k ? jk : jv;
         const bool pre = j < tP;
-        const CUtensorMap* mk = pre ? &p.tm_kp[bl] : &p.tm_ks[bl];
-        const CUtensorMap* mv = pre ? &p.tm_vp[bl] : &p.tm_vs[bl];
         const int key0 = (pre ? j : j - tP) * kBlockN;
-        const uint32_t k_dst = sbase + L::kK + s * L::kKVBytes;
-        const uint32_t v_dst = sbase + L::kV + s * L::kKVBytes;
-        skptx::mbar_arrive_expect_tx(bar(L::bKFull + s), L::kKVBytes);
+        if (do_k) {
+          const int s = j % kKStages;
+          if (j >= kKStages && !W.wait(bar(L::bKEmpty + s), ((j / kKStages) - 1) & 1)) { ok = false; break; }
+          const CUtensorMap* mk = pre ? &p.tm_kp[bl] : &p.tm_ks[bl];
+          skptx::mbar_arrive_expect_tx(bar(L::bKFull + s), L::kKVTile);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          skptx::tma_load_3d(k_dst + c * L::kSub, mk, bar(L::bKFull + s), c * 64, hkv, key0);
-        skptx::mbar_arrive_expect_tx(bar(L::bVFull + s), L::kKVBytes);
+          for (int c = 0; c < D / 64; ++c)
+            skptx::tma_load_3d(sbase + L::kK + s * L::kKVTile + c * L::kSub, mk, bar(L::bKFull + s), c * 64,
+                               hkv, key0);
+          ++jk;
+        } else {
+          const int s = j % kVStages;
+          if (j >= kVStages && !W.wait(bar(L::bVEmpty + s), ((j / kVStages) - 1) & 1)) { ok = false; break; }
+          const CUtensorMap* mv = pre ? &p.tm_vp[bl] : &p.tm_vs[bl];
+          skptx::mbar_arrive_expect_tx(bar(L::bVFull + s), L::kKVTile);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          skptx::tma_load_3d(v_dst + c * L::kSub, mv, bar(L::bVFull + s), c * 64, hkv, key0);
+          for (int c = 0; c < D / 64; ++c)
+            skptx::tma_load_3d(sbase + L::kV + s * L::kKVTile + c * L::kSub, mv, bar(L::bVFull + s), c * 64,
+                               hkv, key0);
+          ++jv;
+        }
       }
       // Drain: no copy issued by this CTA may still be landing when it exits.
       // On the normal path every wait below has already completed.
-      const Waiter drain{abort_flag, p.status, p.wait_limit_ns};
-      drain.wait(bar(L::bQFull), 0);
-      for (int jj = (j > kStages ? j - kStages : 0); jj < j; ++jj) {
-        const int s = jj % kStages;
-        drain.wait(bar(L::bKFull + s), (jj / kStages) & 1);
-        drain.wait(bar(L::bVFull + s), (jj / kStages) & 1);
-      }
+      W.wait(bar(L::bQFull), 0);
+      for (int j = (jk > kKStages ? jk - kKStages : 0); j < jk; ++j)
+        W.wait(bar(L::bKFull + j % kKStages), (j / kKStages) & 1);
+      for (int j = (jv > kVStages ? jv - kVStages : 0); j < jv; ++j)
+        W.wait(bar(L::bVFull + j % kVStages), (j / kVStages) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = skptx::idesc_bf16_f32(kBlockM, kBlockN, false);
-      constexpr uint32_t idO = skptx::idesc_bf16_f32(kBlockM, D, true);
       const uint32_t sQ = sbase + L::kQ;
-      const uint32_t tO = tmem + 256;
-      bool ok = W.wait(bar(L::bQFull), 0);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          const int s = j % kStages;
-          if (!W.wait(bar(L::bKFull + s), (j / kStages) & 1)) { ok = false; break; }
-          // S_j overwrites the buffer that held P_{j-2}: PV_{j-2} must have finished.
-          if (j >= 2 && !W.wait(bar(L::bOReady), (j - 2) & 1)) { ok = false; break; }
-          skptx::tc_fence_after();
-          const uint32_t sK = sbase + L::kK + s * L::kKVBytes;
-          const uint32_t dS = tmem + static_cast<uint32_t>(j & 1) * 128;
+      bool ok = W.wait(bar(L::bQFull), 0) && W.wait(bar(L::bKFull), 0);
+      if (ok) {
+        skptx::tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k / 4) * L::kSub + (k % 4) * 32;
-            skptx::mma_ss(dS, skptx::sdesc_sw128(sQ + off, 16, 1024),
-                          skptx::sdesc_sw128(sK + off, 16, 1024), idS, k > 0 ? 1u : 0u);
-          }
-          skptx::mma_commit(bar(L::bSFull + (j & 1)));
+        for (int x = 0; x < kTilesPerCta; ++x) {
+          issue_s<D>(tmem + x * 128, sQ + x * L::kQTile, sbase + L::kK);
+          skptx::mma_commit(bar(L::bSFull + x));
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int s = jj % kStages;
-          const int b = jj & 1;
-          if (!W.wait(bar(L::bPFull + b), (jj >> 1) & 1)) { ok = false; break; }
-          if (!W.wait(bar(L::bVFull + s), (jj / kStages) & 1)) { ok = false; break; }
-          skptx::tc_fence_after();
-          const uint32_t sV = sbase + L::kV + s * L::kKVBytes;
-          const uint32_t tP_ = tmem + static_cast<uint32_t>(b) * 128;
+        skptx::mma_commit(bar(L::bKEmpty));
+      }
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int vs = j % kVStages;
+        const uint32_t sV = sbase + L::kV + vs * L::kKVTile;
+        const bool more = j + 1 < n_tiles;
+        const int ks = (j + 1) % kKStages;
+        const uint32_t sK = sbase + L::kK + ks * L::kKVTile;
 #pragma unroll
-          for (int k = 0; k < kBlockN / 16; ++k) {
-            skptx::mma_ts(tO, tP_ + k * 8, skptx::sdesc_sw128(sV + k * 2048, L::kSub, 1024), idO,
-                          (jj > 0 || k > 0) ? 1u : 0u);
+        for (int x = 0; x < kTilesPerCta; ++x) {
+          if (!W.wait(bar(L::bPFull + x), j & 1)) { ok = false; break; }
+          if (x == 0 && !W.wait(bar(L::bVFull + vs), (j / kVStages) & 1)) { ok = false; break; }
+          skptx::tc_fence_after();
+          issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, sV, j > 0);
+          skptx::mma_commit(bar(L::bOReady + x));
+          if (x == kTilesPerCta - 1) skptx::mma_commit(bar(L::bVEmpty + vs));
+          if (more) {
+            if (x == 0 && !W.wait(bar(L::bKFull + ks), ((j + 1) / kKStages) & 1)) { ok = false; break; }
+            // S_X(j+1) overwrites P_X(j): PV_X(j) must have read it.
+            if (!W.wait(bar(L::bOReady + x), j & 1)) { ok = false; break; }
+            skptx::tc_fence_after();
+            issue_s<D>(tmem + x * 128, sQ + x * L::kQTile, sK);
+            skptx::mma_commit(bar(L::bSFull + x));
+            if (x == kTilesPerCta - 1) skptx::mma_commit(bar(L::bKEmpty + ks));
           }
-          skptx::mma_commit(bar(L::bKVEmpty + s));
-          skptx::mma_commit(bar(L::bOReady));
         }
       }
       // Every MMA this thread issued has finished before TMEM is released.
       skptx::mma_commit(bar(L::bMmaDone));
-      const Waiter drain{abort_flag, p.status, p.wait_limit_ns};
-      drain.wait(bar(L::bMmaDone), 0);
+      W.wait(bar(L::bMmaDone), 0);
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int r = threadIdx.x;  // row in tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int x = warp / 4;            // query tile of this warpgroup
+    const int r = threadIdx.x % 128;   // row in tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
+    const uint32_t tS_ = tmem + lane_base + static_cast<uint32_t>(x) * 128;
+    const uint32_t tO = tmem + lane_base + 256 + static_cast<uint32_t>(x) * 128;
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;  // running max of scale*log2(e)*s
-    float l_run = 0.f;        // running sum of exponentials
+    float m_run = 0.f;  // running (possibly stale) max of scale*log2(e)*s
+    float l_run = 0.f;  // running sum of exponentials
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, W.wait(bar(L::bSFull + b), (j >> 1) & 1));
+      ok = __all_sync(0xffffffffu, W.wait(bar(L::bSFull + x), j & 1));
       if (!ok) break;
       skptx::tc_fence_after();
-      const uint32_t tS_ = tmem + lane_base + static_cast<uint32_t>(b) * 128;
       uint32_t u[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) skptx::tmem_ld32(tS_ + c * 32, u[c]);
@@ -289,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
       for (int c = 0; c < 4; ++c) skptx::reg_fence(u[c]);
 
-      const int nvalid = (j < tP) ? min(kBlockN, nkp - j * kBlockN) : min(kBlockN, nks - (j - tP) * kBlockN);
+      const int nvalid = tile_valid(j, tP, nkp, nks);
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(u[c / 32][c % 32]);
@@ -298,62 +347,74 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         for (int c = 0; c < 128; ++c)
           if (c >= nvalid) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      // row max with 8 independent chains
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const float alpha = skptx::ex2_approx(m_run - m_new);
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = skptx::ex2_approx(fmaf(s[c], sl2, -m_new));
+      for (int c = 8; c < 128; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_tile = mx * sl2;
+      float alpha = 1.f;
+      bool raise = false;
+      if (j == 0) {
+        m_run = m_tile;
+      } else if (m_tile > m_run + kRescaleLog2) {
+        alpha = skptx::ex2_approx(m_run - m_tile);
+        m_run = m_tile;
+        raise = true;
+      }
+      const float neg_m = -m_run;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) s[c] = skptx::ex2_approx(fmaf(s[c], sl2, neg_m));
       if (nvalid < kBlockN) {
         // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= nvalid) s[c] = 0.f;
       }
-      float sum = 0.f;
+      float sum8[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) sum += s[c];
+      for (int i = 0; i < 8; ++i) sum8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) sum8[c % 8] += s[c];
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * alpha + sum;
-      m_run = m_new;
-      // P (bf16 pairs) overwrites the first 64 columns of this S buffer.
+      // P (bf16 pairs) overwrites the first 64 columns of this tile's S buffer.
       uint32_t pk[2][32];
 #pragma unroll
       for (int i = 0; i < 64; ++i) pk[i / 32][i % 32] = skptx::pack_bf16x2(s[2 * i], s[2 * i + 1]);
       skptx::tmem_st32(tS_, pk[0]);
       skptx::tmem_st32(tS_ + 32, pk[1]);
 
-      if (j > 0) {
-        // O holds sum over tiles < j; rescale once PV_{j-1} has landed.
-        ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady), (j - 1) & 1));
+      if (__any_sync(0xffffffffu, raise)) {
+        // O holds the sum over tiles < j with the old max; PV_X(j-1) must have landed.
+        ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady + x), (j - 1) & 1));
         if (!ok) break;
         skptx::tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          const uint32_t tO = tmem + lane_base + 256;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            skptx::tmem_ld32(tO + c * 32, o);
-            skptx::tmem_wait_ld();
-            skptx::reg_fence(o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          skptx::tmem_ld32(tO + c * 32, o);
+          skptx::tmem_wait_ld();
+          skptx::reg_fence(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            skptx::tmem_st32(tO + c * 32, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          skptx::tmem_st32(tO + c * 32, o);
         }
       }
       skptx::tmem_wait_st();
       skptx::tc_fence_before();
-      skptx::mbar_arrive(bar(L::bPFull + b));
+      skptx::mbar_arrive(bar(L::bPFull + x));
     }
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady), (n_tiles - 1) & 1));
+    if (ok) ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady + x), (n_tiles - 1) & 1));
     if (ok) {
       skptx::tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      const int row = row0 + r;
+      const int row = row0 + x * kBlockM + r;
       uint16_t* orow = out_bh + static_cast<int64_t>(row) * p.out_ss;
-      const uint32_t tO = tmem + lane_base + 256;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -383,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 
   skptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     skptx::tc_fence_after();
     skptx::tmem_dealloc(tmem, kTmemCols);
   }

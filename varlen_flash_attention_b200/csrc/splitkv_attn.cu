@@ -239,7 +239,7 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
   if ((st = device_setup(&dev, &info)) != SK_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
 
-  const int n_qtiles = (Sq + skattn::kBlockM - 1) / skattn::kBlockM;
+  const int n_qtiles = (Sq + skattn::kRowsPerCta - 1) / skattn::kRowsPerCta;
   for (int b0 = 0; b0 < B; b0 += skattn::kMaxBatch) {
     const int nb = std::min(skattn::kMaxBatch, B - b0);
     skattn::AttnParams prm;
