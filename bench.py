@@ -98,6 +98,7 @@ class ClockSampler:
 
     def __init__(self, device_index):
         self.samples = []
+        self.power_w = []
         self.reasons = set()
         self.max_mhz = None
         self._stop = threading.Event()
@@ -118,6 +119,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.power_w.append(nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 for name, attr in self.REASONS.items():
                     if r & getattr(nv, attr, 0):
@@ -142,7 +144,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                     "samples": len(self.samples)}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "power_w_max": max(self.power_w) if self.power_w else None}
 
 
 def dist_setup(n_gpus):
@@ -165,20 +168,29 @@ def barrier(dist):
         dist.barrier()
 
 
-def max_over_ranks(x, dist):
+def max_over_ranks(x, dist, device="cuda"):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(x, dist):
+def sum_over_ranks(x, dist, device="cuda"):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def combine_ranks(flop_per_step, steps, dt_ms, dist, device="cuda"):
+    """Whole-job throughput: all ranks' FLOPs over the slowest rank's time.
+
+    Returns (slowest time in ms, TFLOP/s)."""
+    dt_max = max_over_ranks(dt_ms, dist, device)
+    total = sum_over_ranks(flop_per_step * steps, dist, device)
+    return dt_max, total / (dt_max / 1e3) / 1e12
 
 
 def cpu_oracle_sample(w, target_s=10.0, seed=0):
@@ -290,9 +302,8 @@ def run_ours(args, w):
     status = sk.sk_device_status(local, clear=True)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
-    dt_ms_max = max_over_ranks(dt_ms, dist)
     fl = flops_of(w)
-    value = sum_over_ranks(fl * args.steps, dist) / (dt_ms_max / 1e3) / 1e12
+    dt_ms_max, value = combine_ranks(fl, args.steps, dt_ms, dist)
     per_launch_ms = dt_ms / args.steps
     achieved = fl / (per_launch_ms / 1e3) / 1e12
 
@@ -321,8 +332,7 @@ def run_ours(args, w):
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(dist)
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dist)
-    e2e_value = sum_over_ranks(fl * args.steps, dist) / (e2e_ms / 1e3) / 1e12
+    _, e2e_value = combine_ranks(fl, args.steps, ev0.elapsed_time(ev1), dist)
 
     peak, peak_kind = measured_peaks()
     clocks = clk.summary()

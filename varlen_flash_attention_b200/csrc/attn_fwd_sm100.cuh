@@ -21,9 +21,9 @@
 //              over the first 64 columns of the tile's S buffer.
 //   warp 8     TMA producer: both Q tiles once, then K and V tiles into rings.
 //   warp 9     TMEM allocator + single-thread tcgen05.mma issuer.  Two
-//              independent chains, S_X(j) -> softmax_X(j) -> PV_X(j) ->
-//              S_X(j+1) for X in {A, B}, interleave on the tensor pipe so one
-//              tile's softmax overlaps the other tile's MMAs.
+//              chains, S_X(j) -> softmax_X(j) -> PV_X(j) -> S_X(j+1) for
+//              X in {A, B}, are issued alternately so one tile's softmax
+//              overlaps the other tile's MMAs.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
 // Every wait is bounded (globaltimer); on expiry the CTA raises a device
 // status word, drains its own copies, frees TMEM and exits.
@@ -36,15 +36,63 @@
 
 #include "ptx.cuh"
 
+// Build-time switches (defaults are the shipped configuration).
+#ifndef SKA_SAFE_ALIAS
+#define SKA_SAFE_ALIAS 1   // wait for PV_X(j) to finish before S_X(j+1) overwrites P_X(j)
+#endif
+#ifndef SKA_POLY_EVERY
+#define SKA_POLY_EVERY 0   // k > 0: every k-th score column takes exp2 on the FMA pipe
+#endif
+#ifndef SKA_KSTAGES
+#define SKA_KSTAGES 2
+#endif
+#ifndef SKA_MAX3
+#define SKA_MAX3 0         // three-input max for the row max
+#endif
+#ifndef SKA_SETMAXNREG
+#define SKA_SETMAXNREG 0   // 3 full warpgroups; softmax warps take 224 registers
+#endif
+
+#ifndef SKA_TRACE
+#define SKA_TRACE 0        // record an event timeline of one CTA (profiling builds only)
+#endif
+#ifndef SKA_WAIT_HINT_NS
+#define SKA_WAIT_HINT_NS 0 // > 0: mbarrier waits ask to be suspended up to this long
+#endif
+#ifndef SKA_CHUNKED_P
+#define SKA_CHUNKED_P 0    // exponentiate, pack and store P in 32-column chunks
+#endif
+
 namespace skattn {
+
+#if SKA_TRACE
+// Event timeline of CTA (SKA_TRACE_CTA, 0, 0): per role, entries of
+// code << 56 | tile << 40 | (clock64 & 2^40-1).
+#ifndef SKA_TRACE_CTA
+#define SKA_TRACE_CTA 1
+#endif
+constexpr int kTraceLen = 8192;
+__device__ unsigned long long g_trace[8][kTraceLen];
+__device__ __forceinline__ void trace(int role, int& idx, int code, int j) {
+  if (blockIdx.x == SKA_TRACE_CTA && blockIdx.y == 0 && blockIdx.z == 0 && idx < kTraceLen)
+    g_trace[role][idx++] = (static_cast<unsigned long long>(code) << 56) |
+                           (static_cast<unsigned long long>(j & 0xFFFF) << 40) |
+                           (static_cast<unsigned long long>(clock64()) & 0xFFFFFFFFFFull);
+}
+#define SKA_TR(role, code, j) trace(role, tr_idx, code, j)
+#else
+#define SKA_TR(role, code, j) ((void)0)
+#endif
 
 constexpr int kBlockM = 128;     // query rows per tile
 constexpr int kTilesPerCta = 2;  // query tiles per CTA
 constexpr int kRowsPerCta = kBlockM * kTilesPerCta;
 constexpr int kBlockN = 128;     // keys per KV tile
 constexpr int kMaxBatch = 8;     // batch rows per launch (tensor maps live in parameter space)
-constexpr int kThreads = 320;
-constexpr int kKStages = 2;      // K smem ring depth
+constexpr int kThreads = SKA_SETMAXNREG ? 384 : 320;
+constexpr int kRegsSoftmax = 224;  // per thread after setmaxnreg (softmax warpgroups)
+constexpr int kRegsOther = 56;     // per thread after setmaxnreg (producer / MMA warpgroup)
+constexpr int kKStages = SKA_KSTAGES;  // K smem ring depth
 constexpr int kVStages = 2;      // V smem ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr int32_t kStatusTimeout = 4;
@@ -108,7 +156,11 @@ struct Waiter {
     const uint64_t t0 = skptx::globaltimer_ns();
     uint32_t it = 0;
     while (true) {
+#if SKA_WAIT_HINT_NS > 0
+      if (skptx::mbar_try_wait_hint(bar, parity, SKA_WAIT_HINT_NS)) return true;
+#else
       if (skptx::mbar_try_wait(bar, parity)) return true;
+#endif
       if ((++it & 63u) == 0) {
         if (*abort_flag) return false;
         if (skptx::globaltimer_ns() - t0 > limit_ns) {
@@ -132,31 +184,76 @@ __device__ __forceinline__ void store_zero_rows(uint16_t* base, int64_t ss, int 
   }
 }
 
+// 2^x on the FMA pipe (offloads the MUFU unit).  Cody-Waite split
+// x = n + f, n = nearest integer (added and removed through 1.5 * 2^23),
+// f in [-1/2, 1/2]; p(f) ~= 2^f is the degree-3 minimax polynomial on that
+// interval (relative error 7.5e-5, below the bf16 rounding P gets anyway),
+// coefficients from exp2_poly_fit.py; 2^n is added to p's exponent field.
+// x is clamped at -126 (results there are below 2^-125, i.e. zero for P).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float n = t - 12582912.0f;
+  const float f = x - n;
+  float p = fmaf(0.0551716685f, f, 0.2426111251f);
+  p = fmaf(p, f, 0.6932609677f);
+  p = fmaf(p, f, 0.9999280572f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Valid keys in KV tile j (prefix tiles first, then suffix tiles).
 __device__ __forceinline__ int tile_valid(int j, int tP, int nkp, int nks) {
   return (j < tP) ? min(kBlockN, nkp - j * kBlockN) : min(kBlockN, nks - (j - tP) * kBlockN);
 }
 
+// Descriptor arithmetic: a shared-memory matrix descriptor holds (address >> 4)
+// in its low 14 bits; every operand here lies below 228 KB, so advancing an
+// operand by `bytes` is a plain add of bytes >> 4 (no carry leaves the field).
+// The issue loops below therefore do one add per MMA on precomputed bases.
+
+// S = Q K^T: 128 x 128 x D, both operands K-major, 128-byte swizzle; the
+// K-loop walks 16 columns (32 B) inside a 64-column sub-tile, then the next one.
+#if SKA_TRACE > 1
+#define SKA_TR_MMA(code, k) do { if (tr_idx_p) trace(tr_role, *tr_idx_p, (code) + (k), tr_j); } while (0)
+#define SKA_TR_ARGS , int tr_role = 0, int* tr_idx_p = nullptr, int tr_j = 0
+#else
+#define SKA_TR_MMA(code, k) ((void)0)
+#define SKA_TR_ARGS
+#endif
+
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t sQ, uint32_t sK) {
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc SKA_TR_ARGS) {
   using L = SmemLayout<D>;
   constexpr uint32_t idS = skptx::idesc_bf16_f32(kBlockM, kBlockN, false);
 #pragma unroll
   for (int k = 0; k < D / 16; ++k) {
-    const uint32_t off = (k / 4) * L::kSub + (k % 4) * 32;
-    skptx::mma_ss(d_tmem, skptx::sdesc_sw128(sQ + off, 16, 1024), skptx::sdesc_sw128(sK + off, 16, 1024),
-                  idS, k > 0 ? 1u : 0u);
+    const uint64_t off = ((k / 4) * L::kSub + (k % 4) * 32) >> 4;
+    skptx::mma_ss(d_tmem, q_desc + off, k_desc + off, idS, k > 0 ? 1u : 0u);
+    SKA_TR_MMA(60, k);
   }
 }
 
+// O += P V: P (128 x 128 bf16) from TMEM, V MN-major (head_dim contiguous);
+// each K step covers 16 keys = 2048 B of V rows.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t sV, bool accumulate) {
-  using L = SmemLayout<D>;
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc, bool accumulate SKA_TR_ARGS) {
   constexpr uint32_t idO = skptx::idesc_bf16_f32(kBlockM, D, true);
+  if (accumulate) {
 #pragma unroll
-  for (int k = 0; k < kBlockN / 16; ++k) {
-    skptx::mma_ts(o_tmem, p_tmem + k * 8, skptx::sdesc_sw128(sV + k * 2048, L::kSub, 1024), idO,
-                  (accumulate || k > 0) ? 1u : 0u);
+    for (int k = 0; k < kBlockN / 16; ++k) {
+      skptx::mma_ts(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, 1u);
+      SKA_TR_MMA(50, k);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kBlockN / 16; ++k)
+      skptx::mma_ts(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, k > 0 ? 1u : 0u);
   }
 }
 
@@ -220,9 +317,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   skptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
+#if SKA_TRACE
+  int tr_idx = 0;
+#endif
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
+#if SKA_SETMAXNREG
+    skptx::setmaxnreg_dec<kRegsOther>();
+#endif
     if (lane == 0) {
       const int hkv = hq / p.group;
       skptx::prefetch_tmap(&p.tm_q[bl]);
@@ -246,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (do_k) {
           const int s = j % kKStages;
           if (j >= kKStages && !W.wait(bar(L::bKEmpty + s), ((j / kKStages) - 1) & 1)) { ok = false; break; }
+          SKA_TR(1, 42, j);
           const CUtensorMap* mk = pre ? &p.tm_kp[bl] : &p.tm_ks[bl];
           skptx::mbar_arrive_expect_tx(bar(L::bKFull + s), L::kKVTile);
 #pragma unroll
@@ -256,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         } else {
           const int s = j % kVStages;
           if (j >= kVStages && !W.wait(bar(L::bVEmpty + s), ((j / kVStages) - 1) & 1)) { ok = false; break; }
+          SKA_TR(1, 43, j);
           const CUtensorMap* mv = pre ? &p.tm_vp[bl] : &p.tm_vs[bl];
           skptx::mbar_arrive_expect_tx(bar(L::bVFull + s), L::kKVTile);
 #pragma unroll
@@ -275,39 +380,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    // One thread issues both chains in the order PV_A(j), S_A(j+1), PV_B(j),
+    // S_B(j+1): this keeps tile B's softmax under tile A's MMAs and vice versa.
+#if SKA_SETMAXNREG
+    skptx::setmaxnreg_dec<kRegsOther>();
+#endif
     if (lane == 0) {
-      const uint32_t sQ = sbase + L::kQ;
+      const uint64_t dQ = skptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
+      const uint64_t dK = skptx::sdesc_sw128(sbase + L::kK, 16, 1024);
+      const uint64_t dV = skptx::sdesc_sw128(sbase + L::kV, L::kSub, 1024);
       bool ok = W.wait(bar(L::bQFull), 0) && W.wait(bar(L::bKFull), 0);
+      SKA_TR(0, 1, 0);
       if (ok) {
         skptx::tc_fence_after();
 #pragma unroll
         for (int x = 0; x < kTilesPerCta; ++x) {
-          issue_s<D>(tmem + x * 128, sQ + x * L::kQTile, sbase + L::kK);
+          issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dK);
           skptx::mma_commit(bar(L::bSFull + x));
         }
         skptx::mma_commit(bar(L::bKEmpty));
       }
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int vs = j % kVStages;
-        const uint32_t sV = sbase + L::kV + vs * L::kKVTile;
+        const uint64_t dVs = dV + ((vs * L::kKVTile) >> 4);
         const bool more = j + 1 < n_tiles;
         const int ks = (j + 1) % kKStages;
-        const uint32_t sK = sbase + L::kK + ks * L::kKVTile;
+        const uint64_t dKs = dK + ((ks * L::kKVTile) >> 4);
 #pragma unroll
         for (int x = 0; x < kTilesPerCta; ++x) {
+          const int role = x == 0 ? 0 : 4;
+          (void)role;
           if (!W.wait(bar(L::bPFull + x), j & 1)) { ok = false; break; }
+          SKA_TR(role, 10, j);
           if (x == 0 && !W.wait(bar(L::bVFull + vs), (j / kVStages) & 1)) { ok = false; break; }
+          SKA_TR(role, 12, j);
           skptx::tc_fence_after();
-          issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, sV, j > 0);
+#if SKA_TRACE > 1
+          issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, dVs, j > 0, role, &tr_idx, j);
+#else
+          issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, dVs, j > 0);
+#endif
+          SKA_TR(role, 14, j);
           skptx::mma_commit(bar(L::bOReady + x));
           if (x == kTilesPerCta - 1) skptx::mma_commit(bar(L::bVEmpty + vs));
           if (more) {
             if (x == 0 && !W.wait(bar(L::bKFull + ks), ((j + 1) / kKStages) & 1)) { ok = false; break; }
+            SKA_TR(role, 16, j + 1);
+#if SKA_SAFE_ALIAS
             // S_X(j+1) overwrites P_X(j): PV_X(j) must have read it.
             if (!W.wait(bar(L::bOReady + x), j & 1)) { ok = false; break; }
+#endif
+            SKA_TR(role, 18, j);
             skptx::tc_fence_after();
-            issue_s<D>(tmem + x * 128, sQ + x * L::kQTile, sK);
+#if SKA_TRACE > 1
+            issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dKs, role, &tr_idx, j + 1);
+#else
+            issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dKs);
+#endif
             skptx::mma_commit(bar(L::bSFull + x));
+            SKA_TR(role, 20, j + 1);
             if (x == kTilesPerCta - 1) skptx::mma_commit(bar(L::bKEmpty + ks));
           }
         }
@@ -316,8 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::mma_commit(bar(L::bMmaDone));
       W.wait(bar(L::bMmaDone), 0);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
+#if SKA_SETMAXNREG
+    skptx::setmaxnreg_inc<kRegsSoftmax>();
+#endif
     const int x = warp / 4;            // query tile of this warpgroup
     const int r = threadIdx.x % 128;   // row in tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
@@ -330,6 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     for (int j = 0; j < n_tiles; ++j) {
       ok = __all_sync(0xffffffffu, W.wait(bar(L::bSFull + x), j & 1));
       if (!ok) break;
+      const bool trl = SKA_TRACE && lane == 0 && (x == 0 || warp == 4);
+      const int trole = (warp == 0) ? 2 : (warp == 4 ? 3 : 4 + warp);
+      (void)trole;
+      if (trl) SKA_TR(trole, 30, j);
       skptx::tc_fence_after();
       uint32_t u[4][32];
 #pragma unroll
@@ -337,6 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) skptx::reg_fence(u[c]);
+      if (trl) SKA_TR(trole, 31, j);
 
       const int nvalid = tile_valid(j, tP, nkp, nks);
       float s[128];
@@ -351,8 +490,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#if SKA_MAX3
+#pragma unroll
+      for (int c = 8; c < 120; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[120 + i]);
+#else
 #pragma unroll
       for (int c = 8; c < 128; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], s[c]);
+#endif
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * sl2;
@@ -366,8 +514,46 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         raise = true;
       }
       const float neg_m = -m_run;
+#if SKA_CHUNKED_P
+      // exp2, row sum, bf16 pack and TMEM store in 32-column chunks, so packing
+      // and stores overlap the MUFU-bound exponentials.
+      float sum8[8];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = skptx::ex2_approx(fmaf(s[c], sl2, neg_m));
+      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
+      const bool partial = nvalid < kBlockN;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int c = 32 * ch + i;
+          const float xe = fmaf(s[c], sl2, neg_m);
+          float e;
+          if (SKA_POLY_EVERY > 0 && (c % (SKA_POLY_EVERY > 0 ? SKA_POLY_EVERY : 1)) == SKA_POLY_EVERY - 1)
+            e = exp2_poly(xe);
+          else
+            e = skptx::ex2_approx(xe);
+          // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
+          if (partial && c >= nvalid) e = 0.f;
+          s[c] = e;
+          sum8[i % 8] += e;
+        }
+        uint32_t pk16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk16[i] = skptx::pack_bf16x2(s[32 * ch + 2 * i], s[32 * ch + 2 * i + 1]);
+        skptx::tmem_st16(tS_ + 16 * ch, pk16);
+      }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      l_run = l_run * alpha + sum;
+      if (trl) SKA_TR(trole, 32, j);
+#else
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const float xe = fmaf(s[c], sl2, neg_m);
+        if (SKA_POLY_EVERY > 0 && (c % (SKA_POLY_EVERY > 0 ? SKA_POLY_EVERY : 1)) == SKA_POLY_EVERY - 1)
+          s[c] = exp2_poly(xe);
+        else
+          s[c] = skptx::ex2_approx(xe);
+      }
       if (nvalid < kBlockN) {
         // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
 #pragma unroll
@@ -381,6 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int c = 8; c < 128; ++c) sum8[c % 8] += s[c];
       const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * alpha + sum;
+      if (trl) SKA_TR(trole, 32, j);
       // P (bf16 pairs) overwrites the first 64 columns of this tile's S buffer.
       uint32_t pk[2][32];
 #pragma unroll
@@ -388,6 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::tmem_st32(tS_, pk[0]);
       skptx::tmem_st32(tS_ + 32, pk[1]);
 
+#endif
       if (__any_sync(0xffffffffu, raise)) {
         // O holds the sum over tiles < j with the old max; PV_X(j-1) must have landed.
         ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady + x), (j - 1) & 1));
@@ -407,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::tmem_wait_st();
       skptx::tc_fence_before();
       skptx::mbar_arrive(bar(L::bPFull + x));
+      if (trl) SKA_TR(trole, 35, j);
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady + x), (n_tiles - 1) & 1));
@@ -441,6 +630,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
     }
   }
+
+#if SKA_SETMAXNREG
+  else {
+    skptx::setmaxnreg_dec<kRegsOther>();  // idle warps complete the third warpgroup
+  }
+#endif
 
   skptx::tc_fence_before();
   __syncthreads();
