@@ -17,13 +17,17 @@
 //              softmax in fp32 with exp2 (scale*log2 e folded in); the running
 //              max is only raised when a tile's max exceeds it by more than
 //              kRescaleLog2 (then O and l are rescaled), so most tiles skip the
-//              O round trip through registers.  P goes back to TMEM as bf16,
-//              over the first 64 columns of the tile's S buffer.
+//              O round trip through registers.  P goes back to TMEM as bf16
+//              over the first 64 columns of the tile's S buffer, in 32-column
+//              chunks as soon as each chunk is exponentiated.
 //   warp 8     TMA producer: both Q tiles once, then K and V tiles into rings.
-//   warp 9     TMEM allocator + single-thread tcgen05.mma issuer.  Two
-//              chains, S_X(j) -> softmax_X(j) -> PV_X(j) -> S_X(j+1) for
-//              X in {A, B}, are issued alternately so one tile's softmax
-//              overlaps the other tile's MMAs.
+//   warp 9     TMEM allocator + tcgen05.mma issuer.  Two chains,
+//              S_X(j) -> softmax_X(j) -> PV_X(j) -> S_X(j+1) for X in {A, B},
+//              are issued alternately so one tile's softmax overlaps the other
+//              tile's MMAs.
+// Warps 8 and 9 run their loops warp-convergently (operands stay warp-uniform)
+// and let one elected lane issue each TMA / MMA / commit; a divergent
+// single-lane issuer feeds the tensor pipe measurably slower.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
 // Every wait is bounded (globaltimer); on expiry the CTA raises a device
 // status word, drains its own copies, frees TMEM and exits.
@@ -43,24 +47,11 @@
 #ifndef SKA_POLY_EVERY
 #define SKA_POLY_EVERY 0   // k > 0: every k-th score column takes exp2 on the FMA pipe
 #endif
-#ifndef SKA_KSTAGES
-#define SKA_KSTAGES 2
-#endif
-#ifndef SKA_MAX3
-#define SKA_MAX3 0         // three-input max for the row max
-#endif
-#ifndef SKA_SETMAXNREG
-#define SKA_SETMAXNREG 0   // 3 full warpgroups; softmax warps take 224 registers
-#endif
-
 #ifndef SKA_TRACE
 #define SKA_TRACE 0        // record an event timeline of one CTA (profiling builds only)
 #endif
 #ifndef SKA_WAIT_HINT_NS
 #define SKA_WAIT_HINT_NS 0 // > 0: mbarrier waits ask to be suspended up to this long
-#endif
-#ifndef SKA_CHUNKED_P
-#define SKA_CHUNKED_P 0    // exponentiate, pack and store P in 32-column chunks
 #endif
 
 namespace skattn {
@@ -71,8 +62,9 @@ namespace skattn {
 #ifndef SKA_TRACE_CTA
 #define SKA_TRACE_CTA 1
 #endif
+constexpr int kTraceRoles = 8;
 constexpr int kTraceLen = 8192;
-__device__ unsigned long long g_trace[8][kTraceLen];
+__device__ unsigned long long g_trace[kTraceRoles][kTraceLen];
 __device__ __forceinline__ void trace(int role, int& idx, int code, int j) {
   if (blockIdx.x == SKA_TRACE_CTA && blockIdx.y == 0 && blockIdx.z == 0 && idx < kTraceLen)
     g_trace[role][idx++] = (static_cast<unsigned long long>(code) << 56) |
@@ -89,10 +81,10 @@ constexpr int kTilesPerCta = 2;  // query tiles per CTA
 constexpr int kRowsPerCta = kBlockM * kTilesPerCta;
 constexpr int kBlockN = 128;     // keys per KV tile
 constexpr int kMaxBatch = 8;     // batch rows per launch (tensor maps live in parameter space)
-constexpr int kThreads = SKA_SETMAXNREG ? 384 : 320;
-constexpr int kRegsSoftmax = 224;  // per thread after setmaxnreg (softmax warpgroups)
-constexpr int kRegsOther = 56;     // per thread after setmaxnreg (producer / MMA warpgroup)
-constexpr int kKStages = SKA_KSTAGES;  // K smem ring depth
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr int kKStages = 2;      // K smem ring depth
 constexpr int kVStages = 2;      // V smem ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr int32_t kStatusTimeout = 4;
@@ -128,13 +120,13 @@ struct SmemLayout {
   static constexpr uint32_t kBar = kV + kVStages * kKVTile;
   // barrier indices
   static constexpr int bQFull = 0;
-  static constexpr int bKFull = 1;                     // + stage
-  static constexpr int bKEmpty = bKFull + kKStages;    // + stage
-  static constexpr int bVFull = bKEmpty + kKStages;    // + stage
-  static constexpr int bVEmpty = bVFull + kVStages;    // + stage
-  static constexpr int bSFull = bVEmpty + kVStages;    // + tile
-  static constexpr int bPFull = bSFull + kTilesPerCta; // + tile
-  static constexpr int bOReady = bPFull + kTilesPerCta;// + tile
+  static constexpr int bKFull = 1;                      // + stage
+  static constexpr int bKEmpty = bKFull + kKStages;     // + stage
+  static constexpr int bVFull = bKEmpty + kKStages;     // + stage
+  static constexpr int bVEmpty = bVFull + kVStages;     // + stage
+  static constexpr int bSFull = bVEmpty + kVStages;     // + tile
+  static constexpr int bPFull = bSFull + kTilesPerCta;  // + tile
+  static constexpr int bOReady = bPFull + kTilesPerCta; // + tile
   static constexpr int bMmaDone = bOReady + kTilesPerCta;
   static constexpr int kNumBars = bMmaDone + 1;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
@@ -171,6 +163,11 @@ struct Waiter {
       }
     }
   }
+
+  // Warp-uniform form: every lane waits; true only if all lanes saw the phase.
+  __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity) const {
+    return __all_sync(0xffffffffu, wait(bar, parity));
+  }
 };
 
 __device__ __forceinline__ void store_zero_rows(uint16_t* base, int64_t ss, int r_begin,
@@ -201,10 +198,10 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
+__device__ __forceinline__ float exp2_col(int c, float x) {
+  if (SKA_POLY_EVERY > 0 && (c % (SKA_POLY_EVERY > 0 ? SKA_POLY_EVERY : 1)) == SKA_POLY_EVERY - 1)
+    return exp2_poly(x);
+  return skptx::ex2_approx(x);
 }
 
 // Valid keys in KV tile j (prefix tiles first, then suffix tiles).
@@ -219,42 +216,60 @@ __device__ __forceinline__ int tile_valid(int j, int tP, int nkp, int nks) {
 
 // S = Q K^T: 128 x 128 x D, both operands K-major, 128-byte swizzle; the
 // K-loop walks 16 columns (32 B) inside a 64-column sub-tile, then the next one.
-#if SKA_TRACE > 1
-#define SKA_TR_MMA(code, k) do { if (tr_idx_p) trace(tr_role, *tr_idx_p, (code) + (k), tr_j); } while (0)
-#define SKA_TR_ARGS , int tr_role = 0, int* tr_idx_p = nullptr, int tr_j = 0
-#else
-#define SKA_TR_MMA(code, k) ((void)0)
-#define SKA_TR_ARGS
-#endif
-
+// Warp-collective (one elected lane issues).
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc SKA_TR_ARGS) {
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
   using L = SmemLayout<D>;
   constexpr uint32_t idS = skptx::idesc_bf16_f32(kBlockM, kBlockN, false);
 #pragma unroll
   for (int k = 0; k < D / 16; ++k) {
     const uint64_t off = ((k / 4) * L::kSub + (k % 4) * 32) >> 4;
-    skptx::mma_ss(d_tmem, q_desc + off, k_desc + off, idS, k > 0 ? 1u : 0u);
-    SKA_TR_MMA(60, k);
+    skptx::mma_ss_elect(d_tmem, q_desc + off, k_desc + off, idS, k > 0 ? 1u : 0u);
   }
 }
 
 // O += P V: P (128 x 128 bf16) from TMEM, V MN-major (head_dim contiguous);
-// each K step covers 16 keys = 2048 B of V rows.
+// each K step covers 16 keys = 2048 B of V rows.  Warp-collective.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc, bool accumulate SKA_TR_ARGS) {
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc, bool accumulate) {
   constexpr uint32_t idO = skptx::idesc_bf16_f32(kBlockM, D, true);
   if (accumulate) {
 #pragma unroll
-    for (int k = 0; k < kBlockN / 16; ++k) {
-      skptx::mma_ts(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, 1u);
-      SKA_TR_MMA(50, k);
-    }
+    for (int k = 0; k < kBlockN / 16; ++k)
+      skptx::mma_ts_elect(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, 1u);
   } else {
 #pragma unroll
     for (int k = 0; k < kBlockN / 16; ++k)
-      skptx::mma_ts(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, k > 0 ? 1u : 0u);
+      skptx::mma_ts_elect(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, k > 0 ? 1u : 0u);
   }
+}
+
+// Exponentiate one tile row (in place), sum it, and store P to TMEM in 32-column
+// chunks.  PARTIAL: columns >= nvalid are masked to exact zeros (only the last
+// tile of each source can be partial; full tiles take the branch-free path).
+template <bool PARTIAL>
+__device__ __forceinline__ float exp_row_store_p(float (&s)[kBlockN], float sl2, float neg_m, int nvalid,
+                                                 uint32_t tP) {
+  float sum8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < kBlockN / 32; ++ch) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int c = 32 * ch + i;
+      float e = exp2_col(c, fmaf(s[c], sl2, neg_m));
+      // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
+      if (PARTIAL && c >= nvalid) e = 0.f;
+      s[c] = e;
+      sum8[i % 8] += e;
+    }
+    uint32_t pk16[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk16[i] = skptx::pack_bf16x2(s[32 * ch + 2 * i], s[32 * ch + 2 * i + 1]);
+    skptx::tmem_st16(tP + 16 * ch, pk16);
+  }
+  return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
 }
 
 template <int D>
@@ -308,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     *abort_flag = 0;
     skptx::fence_mbarrier_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     skptx::tmem_alloc(skptx::smem_addr(tmem_slot), kTmemCols);
     skptx::tmem_relinquish();
   }
@@ -319,155 +334,154 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 #if SKA_TRACE
   int tr_idx = 0;
+  const bool tr_lane = lane == 0;
 #endif
 
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
-#if SKA_SETMAXNREG
-    skptx::setmaxnreg_dec<kRegsOther>();
-#endif
+    const int hkv = hq / p.group;
     if (lane == 0) {
-      const int hkv = hq / p.group;
       skptx::prefetch_tmap(&p.tm_q[bl]);
       if (tP > 0) { skptx::prefetch_tmap(&p.tm_kp[bl]); skptx::prefetch_tmap(&p.tm_vp[bl]); }
       if (tS > 0) { skptx::prefetch_tmap(&p.tm_ks[bl]); skptx::prefetch_tmap(&p.tm_vs[bl]); }
-      skptx::mbar_arrive_expect_tx(bar(L::bQFull), kTilesPerCta * L::kQTile);
+    }
+    __syncwarp();
+    skptx::mbar_arrive_expect_tx_elect(bar(L::bQFull), kTilesPerCta * L::kQTile);
 #pragma unroll
-      for (int x = 0; x < kTilesPerCta; ++x)
+    for (int x = 0; x < kTilesPerCta; ++x)
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        skptx::tma_load_3d_elect(sbase + L::kQ + x * L::kQTile + c * L::kSub, &p.tm_q[bl], bar(L::bQFull),
+                                 c * 64, hq, row0 + x * kBlockM);
+    // K(j) is issued one tile ahead of V(j): S needs K first, PV needs V later.
+    int jk = 0, jv = 0;
+    bool ok = true;
+    while (ok && (jk < n_tiles || jv < n_tiles)) {
+      const bool do_k = jk < n_tiles && jk <= jv + 1;
+      const int j = do_k ? jk : jv;
+      const bool pre = j < tP;
+      const int key0 = (pre ? j : j - tP) * kBlockN;
+      if (do_k) {
+        const int s = j % kKStages;
+        if (j >= kKStages && !W.wait_warp(bar(L::bKEmpty + s), ((j / kKStages) - 1) & 1)) { ok = false; break; }
+#if SKA_TRACE
+        if (tr_lane) SKA_TR(1, 42, j);
+#endif
+        const CUtensorMap* mk = pre ? &p.tm_kp[bl] : &p.tm_ks[bl];
+        skptx::mbar_arrive_expect_tx_elect(bar(L::bKFull + s), L::kKVTile);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          skptx::tma_load_3d(sbase + L::kQ + x * L::kQTile + c * L::kSub, &p.tm_q[bl], bar(L::bQFull),
-                             c * 64, hq, row0 + x * kBlockM);
-      // K(j) is issued one tile ahead of V(j): S needs K first, PV needs V later.
-      int jk = 0, jv = 0;
-      bool ok = true;
-      while (ok && (jk < n_tiles || jv < n_tiles)) {
-        const bool do_k = jk < n_tiles && jk <= jv + 1;
-        const int j = do_k ? jk : jv;
-        const bool pre = j < tP;
-        const int key0 = (pre ? j : j - tP) * kBlockN;
-        if (do_k) {
-          const int s = j % kKStages;
-          if (j >= kKStages && !W.wait(bar(L::bKEmpty + s), ((j / kKStages) - 1) & 1)) { ok = false; break; }
-          SKA_TR(1, 42, j);
-          const CUtensorMap* mk = pre ? &p.tm_kp[bl] : &p.tm_ks[bl];
-          skptx::mbar_arrive_expect_tx(bar(L::bKFull + s), L::kKVTile);
+          skptx::tma_load_3d_elect(sbase + L::kK + s * L::kKVTile + c * L::kSub, mk, bar(L::bKFull + s),
+                                   c * 64, hkv, key0);
+        ++jk;
+      } else {
+        const int s = j % kVStages;
+        if (j >= kVStages && !W.wait_warp(bar(L::bVEmpty + s), ((j / kVStages) - 1) & 1)) { ok = false; break; }
+#if SKA_TRACE
+        if (tr_lane) SKA_TR(1, 43, j);
+#endif
+        const CUtensorMap* mv = pre ? &p.tm_vp[bl] : &p.tm_vs[bl];
+        skptx::mbar_arrive_expect_tx_elect(bar(L::bVFull + s), L::kKVTile);
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            skptx::tma_load_3d(sbase + L::kK + s * L::kKVTile + c * L::kSub, mk, bar(L::bKFull + s), c * 64,
-                               hkv, key0);
-          ++jk;
-        } else {
-          const int s = j % kVStages;
-          if (j >= kVStages && !W.wait(bar(L::bVEmpty + s), ((j / kVStages) - 1) & 1)) { ok = false; break; }
-          SKA_TR(1, 43, j);
-          const CUtensorMap* mv = pre ? &p.tm_vp[bl] : &p.tm_vs[bl];
-          skptx::mbar_arrive_expect_tx(bar(L::bVFull + s), L::kKVTile);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            skptx::tma_load_3d(sbase + L::kV + s * L::kKVTile + c * L::kSub, mv, bar(L::bVFull + s), c * 64,
-                               hkv, key0);
-          ++jv;
-        }
+        for (int c = 0; c < D / 64; ++c)
+          skptx::tma_load_3d_elect(sbase + L::kV + s * L::kKVTile + c * L::kSub, mv, bar(L::bVFull + s),
+                                   c * 64, hkv, key0);
+        ++jv;
       }
-      // Drain: no copy issued by this CTA may still be landing when it exits.
-      // On the normal path every wait below has already completed.
-      W.wait(bar(L::bQFull), 0);
-      for (int j = (jk > kKStages ? jk - kKStages : 0); j < jk; ++j)
-        W.wait(bar(L::bKFull + j % kKStages), (j / kKStages) & 1);
-      for (int j = (jv > kVStages ? jv - kVStages : 0); j < jv; ++j)
-        W.wait(bar(L::bVFull + j % kVStages), (j / kVStages) & 1);
     }
-  } else if (warp == 9) {
+    // Drain: no copy issued by this CTA may still be landing when it exits.
+    // On the normal path every wait below has already completed.
+    W.wait_warp(bar(L::bQFull), 0);
+    for (int j = (jk > kKStages ? jk - kKStages : 0); j < jk; ++j)
+      W.wait_warp(bar(L::bKFull + j % kKStages), (j / kKStages) & 1);
+    for (int j = (jv > kVStages ? jv - kVStages : 0); j < jv; ++j)
+      W.wait_warp(bar(L::bVFull + j % kVStages), (j / kVStages) & 1);
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    // One thread issues both chains in the order PV_A(j), S_A(j+1), PV_B(j),
-    // S_B(j+1): this keeps tile B's softmax under tile A's MMAs and vice versa.
-#if SKA_SETMAXNREG
-    skptx::setmaxnreg_dec<kRegsOther>();
+    // Order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): tile B's softmax runs under
+    // tile A's MMAs and vice versa.
+    const uint64_t dQ = skptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
+    const uint64_t dK = skptx::sdesc_sw128(sbase + L::kK, 16, 1024);
+    const uint64_t dV = skptx::sdesc_sw128(sbase + L::kV, L::kSub, 1024);
+    bool ok = W.wait_warp(bar(L::bQFull), 0) && W.wait_warp(bar(L::bKFull), 0);
+#if SKA_TRACE
+    if (tr_lane) SKA_TR(0, 1, 0);
 #endif
-    if (lane == 0) {
-      const uint64_t dQ = skptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
-      const uint64_t dK = skptx::sdesc_sw128(sbase + L::kK, 16, 1024);
-      const uint64_t dV = skptx::sdesc_sw128(sbase + L::kV, L::kSub, 1024);
-      bool ok = W.wait(bar(L::bQFull), 0) && W.wait(bar(L::bKFull), 0);
-      SKA_TR(0, 1, 0);
-      if (ok) {
-        skptx::tc_fence_after();
+    if (ok) {
+      skptx::tc_fence_after();
 #pragma unroll
-        for (int x = 0; x < kTilesPerCta; ++x) {
-          issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dK);
-          skptx::mma_commit(bar(L::bSFull + x));
-        }
-        skptx::mma_commit(bar(L::bKEmpty));
+      for (int x = 0; x < kTilesPerCta; ++x) {
+        issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dK);
+        skptx::mma_commit_elect(bar(L::bSFull + x));
       }
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int vs = j % kVStages;
-        const uint64_t dVs = dV + ((vs * L::kKVTile) >> 4);
-        const bool more = j + 1 < n_tiles;
-        const int ks = (j + 1) % kKStages;
-        const uint64_t dKs = dK + ((ks * L::kKVTile) >> 4);
-#pragma unroll
-        for (int x = 0; x < kTilesPerCta; ++x) {
-          const int role = x == 0 ? 0 : 4;
-          (void)role;
-          if (!W.wait(bar(L::bPFull + x), j & 1)) { ok = false; break; }
-          SKA_TR(role, 10, j);
-          if (x == 0 && !W.wait(bar(L::bVFull + vs), (j / kVStages) & 1)) { ok = false; break; }
-          SKA_TR(role, 12, j);
-          skptx::tc_fence_after();
-#if SKA_TRACE > 1
-          issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, dVs, j > 0, role, &tr_idx, j);
-#else
-          issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, dVs, j > 0);
-#endif
-          SKA_TR(role, 14, j);
-          skptx::mma_commit(bar(L::bOReady + x));
-          if (x == kTilesPerCta - 1) skptx::mma_commit(bar(L::bVEmpty + vs));
-          if (more) {
-            if (x == 0 && !W.wait(bar(L::bKFull + ks), ((j + 1) / kKStages) & 1)) { ok = false; break; }
-            SKA_TR(role, 16, j + 1);
-#if SKA_SAFE_ALIAS
-            // S_X(j+1) overwrites P_X(j): PV_X(j) must have read it.
-            if (!W.wait(bar(L::bOReady + x), j & 1)) { ok = false; break; }
-#endif
-            SKA_TR(role, 18, j);
-            skptx::tc_fence_after();
-#if SKA_TRACE > 1
-            issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dKs, role, &tr_idx, j + 1);
-#else
-            issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dKs);
-#endif
-            skptx::mma_commit(bar(L::bSFull + x));
-            SKA_TR(role, 20, j + 1);
-            if (x == kTilesPerCta - 1) skptx::mma_commit(bar(L::bKEmpty + ks));
-          }
-        }
-      }
-      // Every MMA this thread issued has finished before TMEM is released.
-      skptx::mma_commit(bar(L::bMmaDone));
-      W.wait(bar(L::bMmaDone), 0);
+      skptx::mma_commit_elect(bar(L::bKEmpty));
     }
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ softmax / epilogue
-#if SKA_SETMAXNREG
-    skptx::setmaxnreg_inc<kRegsSoftmax>();
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      const int vs = j % kVStages;
+      const uint64_t dVs = dV + ((vs * L::kKVTile) >> 4);
+      const bool more = j + 1 < n_tiles;
+      const int ks = (j + 1) % kKStages;
+      const uint64_t dKs = dK + ((ks * L::kKVTile) >> 4);
+#pragma unroll
+      for (int x = 0; x < kTilesPerCta; ++x) {
+#if SKA_TRACE
+        const int role = x == 0 ? 0 : 4;
 #endif
+        if (!W.wait_warp(bar(L::bPFull + x), j & 1)) { ok = false; break; }
+#if SKA_TRACE
+        if (tr_lane) SKA_TR(role, 10, j);
+#endif
+        if (x == 0 && !W.wait_warp(bar(L::bVFull + vs), (j / kVStages) & 1)) { ok = false; break; }
+        skptx::tc_fence_after();
+        issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, dVs, j > 0);
+#if SKA_TRACE
+        if (tr_lane) SKA_TR(role, 14, j);
+#endif
+        skptx::mma_commit_elect(bar(L::bOReady + x));
+        if (x == kTilesPerCta - 1) skptx::mma_commit_elect(bar(L::bVEmpty + vs));
+        if (more) {
+          if (x == 0 && !W.wait_warp(bar(L::bKFull + ks), ((j + 1) / kKStages) & 1)) { ok = false; break; }
+#if SKA_SAFE_ALIAS
+          // S_X(j+1) overwrites P_X(j): PV_X(j) must have read it.
+          if (!W.wait_warp(bar(L::bOReady + x), j & 1)) { ok = false; break; }
+#endif
+#if SKA_TRACE
+          if (tr_lane) SKA_TR(role, 18, j);
+#endif
+          skptx::tc_fence_after();
+          issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dKs);
+          skptx::mma_commit_elect(bar(L::bSFull + x));
+#if SKA_TRACE
+          if (tr_lane) SKA_TR(role, 20, j + 1);
+#endif
+          if (x == kTilesPerCta - 1) skptx::mma_commit_elect(bar(L::bKEmpty + ks));
+        }
+      }
+    }
+    // Every MMA this warp issued has finished before TMEM is released.
+    skptx::mma_commit_elect(bar(L::bMmaDone));
+    W.wait_warp(bar(L::bMmaDone), 0);
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
     const int x = warp / 4;            // query tile of this warpgroup
     const int r = threadIdx.x % 128;   // row in tile == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const uint32_t tS_ = tmem + lane_base + static_cast<uint32_t>(x) * 128;
     const uint32_t tO = tmem + lane_base + 256 + static_cast<uint32_t>(x) * 128;
     const float sl2 = p.scale_log2;
+#if SKA_TRACE
+    const bool trl = lane == 0 && (warp % 4) == 0;
+    const int trole = 2 + x;
+#endif
     float m_run = 0.f;  // running (possibly stale) max of scale*log2(e)*s
     float l_run = 0.f;  // running sum of exponentials
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      ok = __all_sync(0xffffffffu, W.wait(bar(L::bSFull + x), j & 1));
+      ok = W.wait_warp(bar(L::bSFull + x), j & 1);
       if (!ok) break;
-      const bool trl = SKA_TRACE && lane == 0 && (x == 0 || warp == 4);
-      const int trole = (warp == 0) ? 2 : (warp == 4 ? 3 : 4 + warp);
-      (void)trole;
+#if SKA_TRACE
       if (trl) SKA_TR(trole, 30, j);
+#endif
       skptx::tc_fence_after();
       uint32_t u[4][32];
 #pragma unroll
@@ -475,32 +489,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) skptx::reg_fence(u[c]);
+#if SKA_TRACE
       if (trl) SKA_TR(trole, 31, j);
-
+#endif
       const int nvalid = tile_valid(j, tP, nkp, nks);
-      float s[128];
+      const bool partial = nvalid < kBlockN;
+      float s[kBlockN];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(u[c / 32][c % 32]);
-      if (nvalid < kBlockN) {
+      for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(u[c / 32][c % 32]);
+      if (partial) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < kBlockN; ++c)
           if (c >= nvalid) s[c] = -INFINITY;
       }
       // row max with 8 independent chains
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = s[i];
-#if SKA_MAX3
 #pragma unroll
-      for (int c = 8; c < 120; c += 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[120 + i]);
-#else
-#pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], s[c]);
-#endif
+      for (int c = 8; c < kBlockN; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], s[c]);
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * sl2;
@@ -513,72 +520,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         m_run = m_tile;
         raise = true;
       }
-      const float neg_m = -m_run;
-#if SKA_CHUNKED_P
-      // exp2, row sum, bf16 pack and TMEM store in 32-column chunks, so packing
-      // and stores overlap the MUFU-bound exponentials.
-      float sum8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
-      const bool partial = nvalid < kBlockN;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c = 32 * ch + i;
-          const float xe = fmaf(s[c], sl2, neg_m);
-          float e;
-          if (SKA_POLY_EVERY > 0 && (c % (SKA_POLY_EVERY > 0 ? SKA_POLY_EVERY : 1)) == SKA_POLY_EVERY - 1)
-            e = exp2_poly(xe);
-          else
-            e = skptx::ex2_approx(xe);
-          // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
-          if (partial && c >= nvalid) e = 0.f;
-          s[c] = e;
-          sum8[i % 8] += e;
-        }
-        uint32_t pk16[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk16[i] = skptx::pack_bf16x2(s[32 * ch + 2 * i], s[32 * ch + 2 * i + 1]);
-        skptx::tmem_st16(tS_ + 16 * ch, pk16);
-      }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      // exp2, row sum, P (bf16 pairs) over the first 64 columns of this S buffer
+      const float sum = partial ? exp_row_store_p<true>(s, sl2, -m_run, nvalid, tS_)
+                                : exp_row_store_p<false>(s, sl2, -m_run, nvalid, tS_);
       l_run = l_run * alpha + sum;
+#if SKA_TRACE
       if (trl) SKA_TR(trole, 32, j);
-#else
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float xe = fmaf(s[c], sl2, neg_m);
-        if (SKA_POLY_EVERY > 0 && (c % (SKA_POLY_EVERY > 0 ? SKA_POLY_EVERY : 1)) == SKA_POLY_EVERY - 1)
-          s[c] = exp2_poly(xe);
-        else
-          s[c] = skptx::ex2_approx(xe);
-      }
-      if (nvalid < kBlockN) {
-        // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= nvalid) s[c] = 0.f;
-      }
-      float sum8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = s[i];
-#pragma unroll
-      for (int c = 8; c < 128; ++c) sum8[c % 8] += s[c];
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-      l_run = l_run * alpha + sum;
-      if (trl) SKA_TR(trole, 32, j);
-      // P (bf16 pairs) overwrites the first 64 columns of this tile's S buffer.
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int i = 0; i < 64; ++i) pk[i / 32][i % 32] = skptx::pack_bf16x2(s[2 * i], s[2 * i + 1]);
-      skptx::tmem_st32(tS_, pk[0]);
-      skptx::tmem_st32(tS_ + 32, pk[1]);
-
 #endif
       if (__any_sync(0xffffffffu, raise)) {
         // O holds the sum over tiles < j with the old max; PV_X(j-1) must have landed.
-        ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady + x), (j - 1) & 1));
+        ok = W.wait_warp(bar(L::bOReady + x), (j - 1) & 1);
         if (!ok) break;
         skptx::tc_fence_after();
 #pragma unroll
@@ -595,10 +546,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::tmem_wait_st();
       skptx::tc_fence_before();
       skptx::mbar_arrive(bar(L::bPFull + x));
+#if SKA_TRACE
       if (trl) SKA_TR(trole, 35, j);
+#endif
     }
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, W.wait(bar(L::bOReady + x), (n_tiles - 1) & 1));
+    if (ok) ok = W.wait_warp(bar(L::bOReady + x), (n_tiles - 1) & 1);
     if (ok) {
       skptx::tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -631,15 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
   }
 
-#if SKA_SETMAXNREG
-  else {
-    skptx::setmaxnreg_dec<kRegsOther>();  // idle warps complete the third warpgroup
-  }
-#endif
-
   skptx::tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     skptx::tc_fence_after();
     skptx::tmem_dealloc(tmem, kTmemCols);
   }

@@ -185,16 +185,6 @@ sk_status_t launch_attn(const skattn::AttnParams& prm, int n_qtiles, int H, int 
     cudaError_t e = cudaFuncSetAttribute(skattn::attn_fwd_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-#if SKA_SETMAXNREG
-    // The warpgroups' register shares after setmaxnreg must fit in what the CTA is
-    // launched with, or setmaxnreg.inc would never complete.
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, skattn::attn_fwd_kernel<D>);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-    const long need = 256L * skattn::kRegsSoftmax + (skattn::kThreads - 256L) * skattn::kRegsOther;
-    if (static_cast<long>(fa.numRegs) * skattn::kThreads < need)
-      return fail(SK_ERR_UNSUPPORTED, "kernel built with %d registers/thread; register split needs %ld", fa.numRegs, need);
-#endif
     dev->attn_attr_set[slot] = true;
   }
   dim3 grid(n_qtiles, H, nb);
@@ -423,7 +413,7 @@ int32_t sk_abi_version(void) { return kAbiVersion; }
 // Profiling builds only: copy the event timeline of the traced CTA to the host.
 SK_API int32_t sk_debug_trace(unsigned long long* host, int32_t n) {
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  const size_t bytes = sizeof(unsigned long long) * std::min<size_t>(n, 5 * skattn::kTraceLen);
+  const size_t bytes = sizeof(unsigned long long) * std::min<size_t>(n, skattn::kTraceRoles * skattn::kTraceLen);
   if (cudaMemcpyFromSymbol(host, skattn::g_trace, bytes) != cudaSuccess) return -1;
   return 0;
 }
