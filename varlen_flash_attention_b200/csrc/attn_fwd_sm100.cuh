@@ -17,14 +17,18 @@
 //              softmax in fp32 with exp2 (scale*log2 e folded in); the running
 //              max is only raised when a tile's max exceeds it by more than
 //              kRescaleLog2 (then O and l are rescaled), so most tiles skip the
-//              O round trip through registers.  P goes back to TMEM as bf16
-//              over the first 64 columns of the tile's S buffer, in 32-column
-//              chunks as soon as each chunk is exponentiated.
+//              O round trip through registers.  P (bf16) goes to shared memory
+//              in the 128-byte-swizzled K-major layout the PV MMA reads.
 //   warp 8     TMA producer: both Q tiles once, then K and V tiles into rings.
-//   warp 9     TMEM allocator + tcgen05.mma issuer.  Two chains,
-//              S_X(j) -> softmax_X(j) -> PV_X(j) -> S_X(j+1) for X in {A, B},
-//              are issued alternately so one tile's softmax overlaps the other
-//              tile's MMAs.
+//   warp 9     TMEM allocator + tcgen05.mma issuer.
+// Because P does not live in the S columns, S_X(j+1) is issued as soon as the
+// softmax of tile X has read S_X(j) into registers: the next scores are ready
+// when the softmax finishes, so each tile's critical path is its softmax alone
+// and the two tiles' softmaxes and all MMAs overlap.  The issuer polls the
+// four op streams (S_A, S_B, PV_A, PV_B) and issues whichever is ready.
+// With head_dim 128 the two tiles share one P buffer (shared memory is full):
+// softmax B(j) stores P after PV_A(j) has read it, softmax A(j+1) after
+// PV_B(j), which keeps the two tiles half a step apart.
 // Warps 8 and 9 run their loops warp-convergently (operands stay warp-uniform)
 // and let one elected lane issue each TMA / MMA / commit; a divergent
 // single-lane issuer feeds the tensor pipe measurably slower.
@@ -41,14 +45,14 @@
 #include "ptx.cuh"
 
 // Build-time switches (defaults are the shipped configuration).
-#ifndef SKA_SAFE_ALIAS
-#define SKA_SAFE_ALIAS 1   // wait for PV_X(j) to finish before S_X(j+1) overwrites P_X(j)
-#endif
 #ifndef SKA_POLY_EVERY
 #define SKA_POLY_EVERY 0   // k > 0: every k-th score column takes exp2 on the FMA pipe
 #endif
 #ifndef SKA_TRACE
 #define SKA_TRACE 0        // record an event timeline of one CTA (profiling builds only)
+#endif
+#ifndef SKA_ISSUE_SLEEP_NS
+#define SKA_ISSUE_SLEEP_NS 0 // > 0: the MMA issuer naps this long when nothing is ready
 #endif
 #ifndef SKA_WAIT_HINT_NS
 #define SKA_WAIT_HINT_NS 0 // > 0: mbarrier waits ask to be suspended up to this long
@@ -114,19 +118,24 @@ struct SmemLayout {
   static constexpr uint32_t kSub = kBlockM * 128;  // one 64-column (128 B) swizzled sub-tile
   static constexpr uint32_t kQTile = kBlockM * D * 2;
   static constexpr uint32_t kKVTile = kBlockN * D * 2;
+  static constexpr uint32_t kPTile = kBlockM * kBlockN * 2;
+  static constexpr int kPBufs = D == 128 ? 1 : 2;                    // P buffers (shared by both tiles when 1)
   static constexpr uint32_t kQ = 0;                                  // + tile * kQTile
   static constexpr uint32_t kK = kQ + kTilesPerCta * kQTile;         // + stage * kKVTile
   static constexpr uint32_t kV = kK + kKStages * kKVTile;            // + stage * kKVTile
-  static constexpr uint32_t kBar = kV + kVStages * kKVTile;
+  static constexpr uint32_t kP = kV + kVStages * kKVTile;            // + buffer * kPTile
+  static constexpr uint32_t kBar = kP + kPBufs * kPTile;
   // barrier indices
   static constexpr int bQFull = 0;
   static constexpr int bKFull = 1;                      // + stage
   static constexpr int bKEmpty = bKFull + kKStages;     // + stage
   static constexpr int bVFull = bKEmpty + kKStages;     // + stage
   static constexpr int bVEmpty = bVFull + kVStages;     // + stage
-  static constexpr int bSFull = bVEmpty + kVStages;     // + tile
-  static constexpr int bPFull = bSFull + kTilesPerCta;  // + tile
-  static constexpr int bOReady = bPFull + kTilesPerCta; // + tile
+  static constexpr int bSFull = bVEmpty + kVStages;     // + tile: S_X(j) is in TMEM
+  static constexpr int bSFree = bSFull + kTilesPerCta;  // + tile: softmax X has read S_X(j)
+  static constexpr int bPFull = bSFree + kTilesPerCta;  // + tile: P_X(j) is in shared memory
+  static constexpr int bPFree = bPFull + kTilesPerCta;  // shared P buffer: the PV MMA reading it finished
+  static constexpr int bOReady = bPFree + 1;            // + tile: PV_X(j) finished
   static constexpr int bMmaDone = bOReady + kTilesPerCta;
   static constexpr int kNumBars = bMmaDone + 1;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
@@ -134,6 +143,7 @@ struct SmemLayout {
   // +1024 slack to align the dynamic base; at least ~116 KB so one CTA per SM
   // (the CTA allocates all 512 TMEM columns).
   static constexpr uint32_t kAlloc = (kEnd + 1024) > 120 * 1024 ? (kEnd + 1024) : 120 * 1024;
+  static_assert(kAlloc <= 232448, "shared memory per CTA");
 };
 
 // Bounded mbarrier wait shared by all roles.  Returns false on timeout or when
@@ -167,6 +177,17 @@ struct Waiter {
   // Warp-uniform form: every lane waits; true only if all lanes saw the phase.
   __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity) const {
     return __all_sync(0xffffffffu, wait(bar, parity));
+  }
+
+  // Wait for this CTA's own asynchronous work (copies, MMAs) to land before
+  // its shared memory or TMEM is released: ignores the abort flag, still
+  // bounded by the time limit.
+  __device__ __forceinline__ void drain_warp(uint32_t bar, uint32_t parity) const {
+    bool done = skptx::mbar_try_wait(bar, parity);
+    const uint64_t t0 = skptx::globaltimer_ns();
+    while (!done && skptx::globaltimer_ns() - t0 <= limit_ns) done = skptx::mbar_try_wait(bar, parity);
+    if (!done) atomicOr(status, kStatusTimeout);
+    __syncwarp();
   }
 };
 
@@ -228,48 +249,54 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64
   }
 }
 
-// O += P V: P (128 x 128 bf16) from TMEM, V MN-major (head_dim contiguous);
-// each K step covers 16 keys = 2048 B of V rows.  Warp-collective.
+// O += P V: P (128 x 128 bf16, K-major, 128-byte swizzle) and V (MN-major,
+// head_dim contiguous) from shared memory; each K step covers 16 keys: 32 B of
+// a P row and 2048 B of V rows.  Warp-collective.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t v_desc, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint64_t p_desc, uint64_t v_desc, bool accumulate) {
+  using L = SmemLayout<D>;
   constexpr uint32_t idO = skptx::idesc_bf16_f32(kBlockM, D, true);
-  if (accumulate) {
 #pragma unroll
-    for (int k = 0; k < kBlockN / 16; ++k)
-      skptx::mma_ts_elect(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, 1u);
-  } else {
-#pragma unroll
-    for (int k = 0; k < kBlockN / 16; ++k)
-      skptx::mma_ts_elect(o_tmem, p_tmem + k * 8, v_desc + ((k * 2048) >> 4), idO, k > 0 ? 1u : 0u);
+  for (int k = 0; k < kBlockN / 16; ++k) {
+    const uint64_t poff = ((k / 4) * L::kSub + (k % 4) * 32) >> 4;
+    skptx::mma_ss_elect(o_tmem, p_desc + poff, v_desc + ((k * 2048) >> 4), idO,
+                        (accumulate || k > 0) ? 1u : 0u);
   }
 }
 
-// Exponentiate one tile row (in place), sum it, and store P to TMEM in 32-column
-// chunks.  PARTIAL: columns >= nvalid are masked to exact zeros (only the last
-// tile of each source can be partial; full tiles take the branch-free path).
+// Exponentiate one tile row, sum it, and pack P as bf16 pairs.  PARTIAL:
+// columns >= nvalid are exact zeros (only the last tile of each source can be
+// partial; full tiles take the select-free path).
 template <bool PARTIAL>
-__device__ __forceinline__ float exp_row_store_p(float (&s)[kBlockN], float sl2, float neg_m, int nvalid,
-                                                 uint32_t tP) {
+__device__ __forceinline__ float exp_row_pack(const float (&s)[kBlockN], float sl2, float neg_m, int nvalid,
+                                              uint32_t (&pk)[kBlockN / 2]) {
   float sum8[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
 #pragma unroll
-  for (int ch = 0; ch < kBlockN / 32; ++ch) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int c = 32 * ch + i;
-      float e = exp2_col(c, fmaf(s[c], sl2, neg_m));
-      // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
-      if (PARTIAL && c >= nvalid) e = 0.f;
-      s[c] = e;
-      sum8[i % 8] += e;
-    }
-    uint32_t pk16[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) pk16[i] = skptx::pack_bf16x2(s[32 * ch + 2 * i], s[32 * ch + 2 * i + 1]);
-    skptx::tmem_st16(tP + 16 * ch, pk16);
+  for (int c = 0; c < kBlockN; c += 2) {
+    float e0 = exp2_col(c, fmaf(s[c], sl2, neg_m));
+    float e1 = exp2_col(c + 1, fmaf(s[c + 1], sl2, neg_m));
+    // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
+    if (PARTIAL && c >= nvalid) e0 = 0.f;
+    if (PARTIAL && c + 1 >= nvalid) e1 = 0.f;
+    sum8[c % 8] += e0;
+    sum8[(c + 1) % 8] += e1;
+    pk[c / 2] = skptx::pack_bf16x2(e0, e1);
   }
   return ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+}
+
+// Store one P row (128 bf16 = 16 chunks of 16 B) of a K-major 128-byte-swizzled
+// tile: chunk q of row r goes to sub-tile q / 8, position (q % 8) ^ (r % 8).
+__device__ __forceinline__ void store_p_row(uint32_t p_base, int r, const uint32_t (&pk)[kBlockN / 2]) {
+  const uint32_t row = p_base + static_cast<uint32_t>(r) * 128u;
+  const uint32_t sw = static_cast<uint32_t>(r & 7);
+#pragma unroll
+  for (int q = 0; q < kBlockN / 8; ++q) {
+    const uint32_t addr = row + (q / 8) * (kBlockM * 128u) + ((static_cast<uint32_t>(q % 8) ^ sw) << 4);
+    skptx::st_shared_v4(addr, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  }
 }
 
 template <int D>
@@ -316,9 +343,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     for (int x = 0; x < kTilesPerCta; ++x) {
       skptx::mbar_init(bar(L::bSFull + x), 1);
+      skptx::mbar_init(bar(L::bSFree + x), kBlockM);
       skptx::mbar_init(bar(L::bPFull + x), kBlockM);
       skptx::mbar_init(bar(L::bOReady + x), 1);
     }
+    skptx::mbar_init(bar(L::bPFree), 1);
     skptx::mbar_init(bar(L::bMmaDone), 1);
     *abort_flag = 0;
     skptx::fence_mbarrier_init();
@@ -334,7 +363,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
 #if SKA_TRACE
   int tr_idx = 0;
-  const bool tr_lane = lane == 0;
 #endif
 
   if (warp == kTmaWarp) {
@@ -353,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       for (int c = 0; c < D / 64; ++c)
         skptx::tma_load_3d_elect(sbase + L::kQ + x * L::kQTile + c * L::kSub, &p.tm_q[bl], bar(L::bQFull),
                                  c * 64, hq, row0 + x * kBlockM);
-    // K(j) is issued one tile ahead of V(j): S needs K first, PV needs V later.
+    // Load order K0, K1, V0, K2, V1, ...: K(j+1) is needed (by S(j+1)) before V(j).
     int jk = 0, jv = 0;
     bool ok = true;
     while (ok && (jk < n_tiles || jv < n_tiles)) {
@@ -365,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int s = j % kKStages;
         if (j >= kKStages && !W.wait_warp(bar(L::bKEmpty + s), ((j / kKStages) - 1) & 1)) { ok = false; break; }
 #if SKA_TRACE
-        if (tr_lane) SKA_TR(1, 42, j);
+        if (lane == 0) SKA_TR(1, 42, j);
 #endif
         const CUtensorMap* mk = pre ? &p.tm_kp[bl] : &p.tm_ks[bl];
         skptx::mbar_arrive_expect_tx_elect(bar(L::bKFull + s), L::kKVTile);
@@ -378,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int s = j % kVStages;
         if (j >= kVStages && !W.wait_warp(bar(L::bVEmpty + s), ((j / kVStages) - 1) & 1)) { ok = false; break; }
 #if SKA_TRACE
-        if (tr_lane) SKA_TR(1, 43, j);
+        if (lane == 0) SKA_TR(1, 43, j);
 #endif
         const CUtensorMap* mv = pre ? &p.tm_vp[bl] : &p.tm_vs[bl];
         skptx::mbar_arrive_expect_tx_elect(bar(L::bVFull + s), L::kKVTile);
@@ -391,21 +419,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
     // Drain: no copy issued by this CTA may still be landing when it exits.
     // On the normal path every wait below has already completed.
-    W.wait_warp(bar(L::bQFull), 0);
+    W.drain_warp(bar(L::bQFull), 0);
     for (int j = (jk > kKStages ? jk - kKStages : 0); j < jk; ++j)
-      W.wait_warp(bar(L::bKFull + j % kKStages), (j / kKStages) & 1);
+      W.drain_warp(bar(L::bKFull + j % kKStages), (j / kKStages) & 1);
     for (int j = (jv > kVStages ? jv - kVStages : 0); j < jv; ++j)
-      W.wait_warp(bar(L::bVFull + j % kVStages), (j / kVStages) & 1);
+      W.drain_warp(bar(L::bVFull + j % kVStages), (j / kVStages) & 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    // Order PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): tile B's softmax runs under
-    // tile A's MMAs and vice versa.
     const uint64_t dQ = skptx::sdesc_sw128(sbase + L::kQ, 16, 1024);
     const uint64_t dK = skptx::sdesc_sw128(sbase + L::kK, 16, 1024);
     const uint64_t dV = skptx::sdesc_sw128(sbase + L::kV, L::kSub, 1024);
+    const uint64_t dP = skptx::sdesc_sw128(sbase + L::kP, 16, 1024);
     bool ok = W.wait_warp(bar(L::bQFull), 0) && W.wait_warp(bar(L::bKFull), 0);
 #if SKA_TRACE
-    if (tr_lane) SKA_TR(0, 1, 0);
+    if (lane == 0) SKA_TR(0, 1, 0);
 #endif
     if (ok) {
       skptx::tc_fence_after();
@@ -416,51 +443,81 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       }
       skptx::mma_commit_elect(bar(L::bKEmpty));
     }
-    for (int j = 0; ok && j < n_tiles; ++j) {
-      const int vs = j % kVStages;
-      const uint64_t dVs = dV + ((vs * L::kKVTile) >> 4);
-      const bool more = j + 1 < n_tiles;
-      const int ks = (j + 1) % kKStages;
-      const uint64_t dKs = dK + ((ks * L::kKVTile) >> 4);
+    // Each tile has two in-order streams, S_X(1..n-1) and PV_X(0..n-1); any op
+    // whose inputs are ready is issued, so neither tile's progress waits for
+    // the other's.  A K (V) stage is released once both tiles' S (PV) MMAs
+    // reading it are issued (the commit fires when they complete).
+    // Warp-uniform readiness: every lane probes, all must agree (else retry).
+    auto ready = [](uint32_t b, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, skptx::mbar_test_wait(b, parity));
+    };
+    int sN[kTilesPerCta], pN[kTilesPerCta];
+#pragma unroll
+    for (int x = 0; x < kTilesPerCta; ++x) { sN[x] = 1; pN[x] = 0; }
+    uint64_t stall_t0 = 0;
+    uint32_t spins = 0;
+    while (ok && (pN[0] < n_tiles || pN[1] < n_tiles)) {
+      bool progressed = false;
 #pragma unroll
       for (int x = 0; x < kTilesPerCta; ++x) {
+        const int o = 1 - x;
+        const int j = pN[x];
+        if (j < n_tiles && ready(bar(L::bPFull + x), j & 1) &&
+            ready(bar(L::bVFull + j % kVStages), (j / kVStages) & 1)) {
 #if SKA_TRACE
-        const int role = x == 0 ? 0 : 4;
-#endif
-        if (!W.wait_warp(bar(L::bPFull + x), j & 1)) { ok = false; break; }
-#if SKA_TRACE
-        if (tr_lane) SKA_TR(role, 10, j);
-#endif
-        if (x == 0 && !W.wait_warp(bar(L::bVFull + vs), (j / kVStages) & 1)) { ok = false; break; }
-        skptx::tc_fence_after();
-        issue_pv<D>(tmem + 256 + x * 128, tmem + x * 128, dVs, j > 0);
-#if SKA_TRACE
-        if (tr_lane) SKA_TR(role, 14, j);
-#endif
-        skptx::mma_commit_elect(bar(L::bOReady + x));
-        if (x == kTilesPerCta - 1) skptx::mma_commit_elect(bar(L::bVEmpty + vs));
-        if (more) {
-          if (x == 0 && !W.wait_warp(bar(L::bKFull + ks), ((j + 1) / kKStages) & 1)) { ok = false; break; }
-#if SKA_SAFE_ALIAS
-          // S_X(j+1) overwrites P_X(j): PV_X(j) must have read it.
-          if (!W.wait_warp(bar(L::bOReady + x), j & 1)) { ok = false; break; }
-#endif
-#if SKA_TRACE
-          if (tr_lane) SKA_TR(role, 18, j);
+          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 10, j);
 #endif
           skptx::tc_fence_after();
-          issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dKs);
-          skptx::mma_commit_elect(bar(L::bSFull + x));
+          const int b = x % L::kPBufs;
+          issue_pv<D>(tmem + 256 + x * 128, dP + ((b * L::kPTile) >> 4),
+                      dV + (((j % kVStages) * L::kKVTile) >> 4), j > 0);
+          skptx::mma_commit_elect(bar(L::bOReady + x));
+          if (L::kPBufs == 1) skptx::mma_commit_elect(bar(L::bPFree));
+          if (pN[o] > j) skptx::mma_commit_elect(bar(L::bVEmpty + j % kVStages));
+          pN[x] = j + 1;
+          progressed = true;
 #if SKA_TRACE
-          if (tr_lane) SKA_TR(role, 20, j + 1);
+          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 14, j);
 #endif
-          if (x == kTilesPerCta - 1) skptx::mma_commit_elect(bar(L::bKEmpty + ks));
+        }
+        const int k = sN[x];
+        if (k < n_tiles && ready(bar(L::bSFree + x), (k - 1) & 1) &&
+            ready(bar(L::bKFull + k % kKStages), (k / kKStages) & 1)) {
+#if SKA_TRACE
+          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 18, k - 1);
+#endif
+          skptx::tc_fence_after();
+          issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dK + (((k % kKStages) * L::kKVTile) >> 4));
+          skptx::mma_commit_elect(bar(L::bSFull + x));
+          if (sN[o] > k) skptx::mma_commit_elect(bar(L::bKEmpty + k % kKStages));
+          sN[x] = k + 1;
+          progressed = true;
+#if SKA_TRACE
+          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 20, k);
+#endif
         }
       }
+      // Bounded: give up once nothing has become ready for the wait limit.
+      if (progressed) {
+        spins = 0;
+      } else if (spins++ == 0) {
+        stall_t0 = skptx::globaltimer_ns();
+      } else if ((spins & 31u) == 0) {
+        if (*abort_flag) ok = false;
+        else if (skptx::globaltimer_ns() - stall_t0 > p.wait_limit_ns) {
+          *abort_flag = 1;
+          atomicOr(p.status, kStatusTimeout);
+          ok = false;
+        }
+        ok = __all_sync(0xffffffffu, ok);
+      }
+#if SKA_ISSUE_SLEEP_NS > 0
+      if (!progressed) __nanosleep(SKA_ISSUE_SLEEP_NS);
+#endif
     }
     // Every MMA this warp issued has finished before TMEM is released.
     skptx::mma_commit_elect(bar(L::bMmaDone));
-    W.wait_warp(bar(L::bMmaDone), 0);
+    W.drain_warp(bar(L::bMmaDone), 0);
   } else {
     // ------------------------------------------------------------ softmax / epilogue
     const int x = warp / 4;            // query tile of this warpgroup
@@ -468,6 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
     const uint32_t tS_ = tmem + lane_base + static_cast<uint32_t>(x) * 128;
     const uint32_t tO = tmem + lane_base + 256 + static_cast<uint32_t>(x) * 128;
+    const int pb = x % L::kPBufs;
+    const uint32_t p_base = sbase + L::kP + pb * L::kPTile;
     const float sl2 = p.scale_log2;
 #if SKA_TRACE
     const bool trl = lane == 0 && (warp % 4) == 0;
@@ -483,20 +542,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (trl) SKA_TR(trole, 30, j);
 #endif
       skptx::tc_fence_after();
-      uint32_t u[4][32];
+      float s[kBlockN];
+      {
+        uint32_t u[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) skptx::tmem_ld32(tS_ + c * 32, u[c]);
-      skptx::tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) skptx::tmem_ld32(tS_ + c * 32, u[c]);
+        skptx::tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) skptx::reg_fence(u[c]);
+        for (int c = 0; c < 4; ++c) skptx::reg_fence(u[c]);
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(u[c / 32][c % 32]);
+      }
+      // S_X(j) is in registers: the issuer may overwrite it with S_X(j+1).
+      skptx::tc_fence_before();
+      skptx::mbar_arrive(bar(L::bSFree + x));
 #if SKA_TRACE
       if (trl) SKA_TR(trole, 31, j);
 #endif
       const int nvalid = tile_valid(j, tP, nkp, nks);
       const bool partial = nvalid < kBlockN;
-      float s[kBlockN];
-#pragma unroll
-      for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(u[c / 32][c % 32]);
       if (partial) {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
@@ -520,17 +584,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         m_run = m_tile;
         raise = true;
       }
-      // exp2, row sum, P (bf16 pairs) over the first 64 columns of this S buffer
-      const float sum = partial ? exp_row_store_p<true>(s, sl2, -m_run, nvalid, tS_)
-                                : exp_row_store_p<false>(s, sl2, -m_run, nvalid, tS_);
+      uint32_t pk[kBlockN / 2];
+      const float sum = partial ? exp_row_pack<true>(s, sl2, -m_run, nvalid, pk)
+                                : exp_row_pack<false>(s, sl2, -m_run, nvalid, pk);
       l_run = l_run * alpha + sum;
 #if SKA_TRACE
       if (trl) SKA_TR(trole, 32, j);
 #endif
-      if (__any_sync(0xffffffffu, raise)) {
-        // O holds the sum over tiles < j with the old max; PV_X(j-1) must have landed.
+      // Before P_X(j) is stored and before O_X is touched, PV_X(j-1) must have
+      // finished.  This also keeps every barrier below within one phase of
+      // its waiter (a parity wait cannot tell phase k from k+2).
+      if (j > 0) {
         ok = W.wait_warp(bar(L::bOReady + x), (j - 1) & 1);
         if (!ok) break;
+      }
+      if (L::kPBufs == 1) {
+        // One P buffer for both tiles, used in the order A(0), B(0), A(1), ...:
+        // use u may start once the PV MMA of use u-1 has finished.
+        const int use = 2 * j + x;
+        if (use > 0) {
+          ok = W.wait_warp(bar(L::bPFree), (use - 1) & 1);
+          if (!ok) break;
+        }
+      }
+      store_p_row(p_base, r, pk);
+      if (__any_sync(0xffffffffu, raise)) {
+        // O holds the sum over tiles < j with the old max (PV_X(j) waits for
+        // this thread's arrive below).
         skptx::tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -542,8 +622,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           skptx::tmem_st32(tO + c * 32, o);
         }
+        skptx::tmem_wait_st();
       }
-      skptx::tmem_wait_st();
+      skptx::fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
       skptx::tc_fence_before();
       skptx::mbar_arrive(bar(L::bPFull + x));
 #if SKA_TRACE
