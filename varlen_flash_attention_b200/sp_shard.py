@@ -1,0 +1,209 @@
+"""Sequence-parallel shard helpers: even tail-padded shards and the attention
+metadata they imply ("sglang PR 30107", unified SP shard utils).
+
+Layout invariant (same page): a sequence of ``orig_len`` tokens is split into
+``sp_size`` equal chunks of ``local_len = ceil(orig_len / sp_size)`` tokens;
+the ``num_pad = local_len * sp_size - orig_len`` pad tokens all sit at the end
+of the LAST rank's chunk, so the gathered sequence carries one contiguous pad
+block at its global tail.  That is exactly the layout ``attn_fwd_split_kv``
+excludes for free through ``real_len``: after the sequence is gathered (or
+after a Ulysses all-to-all), every rank passes ``real_len = orig_len`` (times
+any per-token row multiplier) and no pad key enters the softmax.
+
+Host-side plumbing only (shape math, ``F.pad``/``narrow``/``cat`` and
+``torch.distributed`` gathers); nothing here is on the attention hot path.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Optional, Sequence, Tuple
+
+import torch
+import torch.nn.functional as F
+
+__all__ = [
+    "SpShard",
+    "build_shard_plan",
+    "tail_attn_meta",
+    "attn_real_len",
+    "shard_like",
+    "shard_seq",
+    "gather_seq",
+    "join_seqs",
+    "split_seqs",
+    "should_shard_text",
+]
+
+
+@dataclass(frozen=True)
+class SpShard:
+    """Facts of one tail-padded even shard, shared by every tensor of a stream."""
+
+    orig_len: int   # real tokens (global)
+    local_len: int  # tokens per rank (equal on every rank)
+    num_pad: int    # pad tokens, all at the global tail (the last rank's chunk end)
+    sp_size: int
+    sp_rank: int
+
+    @property
+    def local_pad(self) -> int:
+        """Pad rows inside this rank's chunk.  Whenever ``num_pad <= local_len``
+        (every case but tiny sequences over many ranks) this is the page's rule,
+        ``num_pad`` on the last rank and 0 elsewhere.  When the pad outnumbers a
+        chunk (e.g. 1 token over 4 ranks: local_len 1, num_pad 3) it spills into
+        earlier chunks and this counts the pad rows actually inside this one,
+        so ``local_real_len`` never goes negative."""
+        end = (self.sp_rank + 1) * self.local_len
+        return max(0, min(self.local_len, end - self.orig_len))
+
+    @property
+    def local_real_len(self) -> int:
+        """Real tokens in this rank's chunk."""
+        return self.local_len - self.local_pad
+
+    @property
+    def padded_len(self) -> int:
+        """Length of the gathered (padded) sequence."""
+        return self.local_len * self.sp_size
+
+
+def _group_size_rank(group) -> Tuple[int, int]:
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return 1, 0
+    return dist.get_world_size(group), dist.get_rank(group)
+
+
+def build_shard_plan(seq_len: int, sp_size: Optional[int] = None, sp_rank: Optional[int] = None,
+                     group=None) -> SpShard:
+    """Shard math only, no tensors ("sglang PR 30107", ``build_shard_plan``):
+    ``local_len = ceil(seq_len / sp_size)``, ``num_pad = local_len * sp_size - seq_len``.
+
+    ``sp_size``/``sp_rank`` default to the size and rank of ``group`` (the
+    default process group), or to (1, 0) when torch.distributed is not
+    initialised.  With ``sp_size == 1`` the plan is the identity.
+    """
+    if sp_size is None or sp_rank is None:
+        gs, gr = _group_size_rank(group)
+        sp_size = gs if sp_size is None else sp_size
+        sp_rank = gr if sp_rank is None else sp_rank
+    if seq_len < 0:
+        raise ValueError(f"seq_len must be >= 0, got {seq_len}")
+    if sp_size < 1 or not (0 <= sp_rank < sp_size):
+        raise ValueError(f"bad sp_size/sp_rank: {sp_size}/{sp_rank}")
+    if sp_size == 1:
+        return SpShard(seq_len, seq_len, 0, 1, 0)
+    local_len = (seq_len + sp_size - 1) // sp_size
+    return SpShard(orig_len=seq_len, local_len=local_len, num_pad=local_len * sp_size - seq_len,
+                   sp_size=sp_size, sp_rank=sp_rank)
+
+
+def tail_attn_meta(shard: SpShard, seqlen_multiplier: int = 1) -> Optional[dict]:
+    """Tail-pad attention metadata of this rank's chunk ("sglang PR 30107",
+    ``tail_attn_meta``): None without pad, else ``valid_len = local_real_len *
+    multiplier`` and ``max_seqlen_tail = max(valid_len, num_pad)`` (the page's
+    fix for the degenerate case where the pad outnumbers the valid tokens).
+    ``seqlen_multiplier`` scales tokens to attention rows (e.g. several rows
+    per token)."""
+    if shard.num_pad == 0:
+        return None
+    valid = shard.local_real_len * seqlen_multiplier
+    return {"tail": True, "valid_len": valid, "max_seqlen_tail": max(valid, shard.num_pad)}
+
+
+def attn_real_len(shard: SpShard, seqlen_multiplier: int = 1, batch: int = 1) -> List[int]:
+    """``real_len`` for ``attn_fwd_split_kv`` over the gathered sequence (pad at
+    the global tail): the valid key count ``orig_len * multiplier`` for each of
+    ``batch`` rows.  The kernel takes no ``max_seqlen``, so the page's
+    ``max_seqlen_tail`` has no counterpart here."""
+    return [shard.orig_len * seqlen_multiplier] * batch
+
+
+def shard_like(x: torch.Tensor, shard: SpShard, dim: int = 1, pad_mode: str = "zeros") -> torch.Tensor:
+    """Apply a planned shard to one tensor ("sglang PR 30107", ``shard_like``):
+    pad the tail of ``dim`` with ``num_pad`` rows (zeros, or copies of the last
+    row with ``pad_mode="repeat_last"``), then take this rank's ``local_len``
+    rows.  Tensors of one stream (hidden states, RoPE tables, ...) sharded
+    with the same plan stay aligned chunk for chunk."""
+    if x.shape[dim] != shard.orig_len:
+        raise ValueError(f"dim {dim} has {x.shape[dim]} rows, plan expects {shard.orig_len}")
+    if shard.sp_size <= 1:
+        return x
+    if shard.num_pad > 0:
+        if pad_mode == "repeat_last":
+            if shard.orig_len == 0:
+                raise ValueError("repeat_last needs at least one row")
+            last = x.narrow(dim, x.shape[dim] - 1, 1)
+            x = torch.cat([x, last.expand(*[shard.num_pad if i == dim else -1 for i in range(x.dim())])], dim=dim)
+        elif pad_mode == "zeros":
+            nd = dim % x.dim()
+            pads = [0, 0] * (x.dim() - 1 - nd) + [0, shard.num_pad]
+            x = F.pad(x, pads)
+        else:
+            raise ValueError(f"unknown pad_mode {pad_mode!r}")
+    return x.narrow(dim, shard.sp_rank * shard.local_len, shard.local_len)
+
+
+def shard_seq(x: torch.Tensor, shard: SpShard, dim: int = 1, pad_mode: str = "zeros") -> torch.Tensor:
+    """This rank's chunk of a full sequence (``shard_like`` under the stream's plan)."""
+    return shard_like(x, shard, dim=dim, pad_mode=pad_mode)
+
+
+def gather_seq(x_local: torch.Tensor, shard: SpShard, dim: int = 1, group=None) -> torch.Tensor:
+    """Inverse of ``shard_seq`` over a process group: all-gather the ranks'
+    chunks along ``dim`` (rank order) and trim the tail pad back to
+    ``orig_len`` rows."""
+    import torch.distributed as dist
+
+    if x_local.shape[dim] != shard.local_len:
+        raise ValueError(f"chunk has {x_local.shape[dim]} rows, plan expects {shard.local_len}")
+    if shard.sp_size <= 1:
+        return x_local
+    xs = x_local.contiguous()
+    parts = [torch.empty_like(xs) for _ in range(shard.sp_size)]
+    dist.all_gather(parts, xs, group=group)
+    return torch.cat(parts, dim=dim).narrow(dim, 0, shard.orig_len)
+
+
+def join_seqs(firsts: Sequence[torch.Tensor], seconds: Sequence[torch.Tensor], local_pad: int,
+              dim: int = 1) -> List[torch.Tensor]:
+    """Joint sequences with the first stream's local pad moved to the joint
+    tail: ``cat([first[:-pad], second, first[-pad:]])`` per tensor pair (e.g.
+    text then image tokens, for q, k and v alike).  The page names this helper
+    and states only that it keeps the pad at the tail; this is that layout."""
+    if len(firsts) != len(seconds):
+        raise ValueError("join_seqs needs tensor pairs")
+    out = []
+    for a, b in zip(firsts, seconds):
+        la = a.shape[dim]
+        if not 0 <= local_pad <= la:
+            raise ValueError(f"local_pad {local_pad} outside [0, {la}]")
+        valid = a.narrow(dim, 0, la - local_pad)
+        pad = a.narrow(dim, la - local_pad, local_pad)
+        out.append(torch.cat([valid, b, pad], dim=dim))
+    return out
+
+
+def split_seqs(joints: Sequence[torch.Tensor], first_len: int, local_pad: int,
+               dim: int = 1) -> List[Tuple[torch.Tensor, torch.Tensor]]:
+    """Inverse of ``join_seqs``: from ``[first valid | second | first pad]``
+    return ``(first, second)`` with the first stream's pad back at its own
+    tail; ``first_len`` counts the first stream's rows including the pad."""
+    out = []
+    for j in joints:
+        n = j.shape[dim]
+        valid = first_len - local_pad
+        second_len = n - first_len
+        if valid < 0 or second_len < 0:
+            raise ValueError("first_len/local_pad do not fit the joint sequence")
+        first = torch.cat([j.narrow(dim, 0, valid), j.narrow(dim, n - local_pad, local_pad)], dim=dim)
+        out.append((first, j.narrow(dim, valid, second_len)))
+    return out
+
+
+def should_shard_text(seq_len: int, sp_size: int, min_len: int = 0) -> bool:
+    """Policy gate: shard a stream across ``sp_size`` ranks unless it is
+    shorter than ``min_len`` tokens (the page's default is to always shard,
+    with an escape hatch for a minimum length)."""
+    return sp_size > 1 and seq_len >= max(min_len, 1)
