@@ -115,6 +115,38 @@ SK_API sk_status_t attn_fwd_split_kv_ex(const sk_tensor_t* q, const sk_tensor_t*
                                  const int32_t* q_valid, void* stream);
 
 /*
+ * attn_fwd_varlen — packed variable-length attention: several independent
+ * sequences (segments) concatenated along one token axis, each attending only
+ * to its own keys (a block-diagonal mask, never materialised).  Sources:
+ * "vLLM-Omni performance patterns" (packed varlen attention driven by
+ * cu_seqlens computed once on the host, validated against dense attention
+ * with unequal sample lengths and padding exclusion) and "sglang PR 30107"
+ * (varlen FlashAttention over [valid | pad] segments).
+ *
+ *   q    [1, Tq, num_q_heads, head_dim]  (read; stride_b ignored)
+ *   k, v [1, Tk, num_kv_heads, head_dim] (read)
+ *   cu_seqlens_q, cu_seqlens_k  HOST int32[num_segments + 1], non-decreasing,
+ *        cu[0] >= 0, cu_q[n] <= Tq, cu_k[n] <= Tk.  Segment i owns query rows
+ *        [cu_q[i], cu_q[i+1]) and key rows [cu_k[i], cu_k[i+1]).
+ *   seqused_q, seqused_k  HOST int32[num_segments] or NULL: the first
+ *        seqused_*[i] rows of segment i are valid (the rest is pad: pad keys
+ *        are never loaded, pad query rows are written as zeros).  NULL = all.
+ *   softmax_scale  finite, >= 0.   head_dim  64 or 128.
+ *   out  [1, Tq, num_q_heads, head_dim] (written on the segments' rows only;
+ *        rows outside every segment are not touched); must not overlap the
+ *        inputs or itself.
+ * A segment with no valid key writes zeros.  One kernel launch per 8
+ * segments, on `stream`.  Returns SK_OK, SK_ERR_INVALID_ARG,
+ * SK_ERR_UNSUPPORTED or SK_ERR_CUDA.
+ */
+SK_API sk_status_t attn_fwd_varlen(const sk_tensor_t* q, const sk_tensor_t* k, const sk_tensor_t* v,
+                                   const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                   const int32_t* seqused_q, const int32_t* seqused_k,
+                                   int32_t num_segments, int32_t num_q_heads, int32_t num_kv_heads,
+                                   float softmax_scale, const sk_tensor_t* out, int32_t head_dim,
+                                   void* stream);
+
+/*
  * qk_rmsnorm_rope — fused Q/K RMSNorm over head_dim followed by rotary
  * embedding, in place on q and k (which may be strided views of one fused
  * QKV buffer).  Source: "vLLM-Omni performance patterns", Q/K RMSNorm + RoPE

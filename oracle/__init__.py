@@ -156,6 +156,45 @@ def attn_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix,
     return out
 
 
+def attn_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int],
+                seqused_q: Optional[Sequence[int]] = None,
+                seqused_k: Optional[Sequence[int]] = None,
+                softmax_scale: Optional[float] = None) -> np.ndarray:
+    """Packed variable-length attention, fp64 ("vLLM-Omni performance
+    patterns": packed samples described by cu_seqlens; "sglang PR 30107":
+    varlen attention over [valid | pad] segments).  The definition is a
+    block-diagonal mask: query row t of segment i attends to the first
+    seqused_k[i] keys of segment i only, i.e. it is single-sequence attention
+    applied to each segment's slices.  Rows past seqused_q[i] inside a segment,
+    and segments without a valid key, give zeros; rows outside every segment
+    are returned as zeros too.
+
+    q [Tq, Hq, D] (or [1, Tq, Hq, D]), k/v [Tk, Hkv, D]; returns float64 [Tq, Hq, D].
+    """
+    import torch
+
+    def as3(t):
+        return t[0] if t.dim() == 4 else t
+
+    q3, k3, v3 = as3(q), as3(k), as3(v)
+    Tq, Hq, D = q3.shape
+    n = len(cu_seqlens_q) - 1
+    out = np.zeros((Tq, Hq, D), dtype=np.float64)
+    empty = k3[:0].unsqueeze(0)
+    for i in range(n):
+        q0, q1 = int(cu_seqlens_q[i]), int(cu_seqlens_q[i + 1])
+        k0, k1 = int(cu_seqlens_k[i]), int(cu_seqlens_k[i + 1])
+        if q1 == q0:
+            continue
+        nk = (k1 - k0) if seqused_k is None else int(seqused_k[i])
+        nq = (q1 - q0) if seqused_q is None else int(seqused_q[i])
+        seg = attn_split_kv(q3[q0:q1].unsqueeze(0), empty, empty,
+                            k3[k0:k1].unsqueeze(0), v3[k0:k1].unsqueeze(0),
+                            real_len=[nk], q_valid=[nq], softmax_scale=softmax_scale)
+        out[q0:q1] = seg[0]
+    return out
+
+
 def qk_rmsnorm_rope(x, w, table, pos=None, rot_dim: Optional[int] = None,
                     interleaved: bool = False, eps: float = 1e-6) -> np.ndarray:
     """RMSNorm over head_dim then RoPE for x [..., H, D] (bf16); returns bf16 bits (uint16).

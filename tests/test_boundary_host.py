@@ -29,7 +29,7 @@ def _declared_symbols():
 
 def test_header_declares_the_entry_points():
     names = set(_declared_symbols())
-    assert {"attn_fwd_split_kv", "attn_fwd_split_kv_ex", "qk_rmsnorm_rope", "sk_last_error",
+    assert {"attn_fwd_split_kv", "attn_fwd_split_kv_ex", "attn_fwd_varlen", "qk_rmsnorm_rope", "sk_last_error",
             "sk_device_status", "sk_set_wait_timeout_ms", "sk_abi_version"} <= names
 
 
@@ -163,3 +163,50 @@ def test_python_binding_raises_on_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sk, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         sk.lib()
+
+
+# ---------------------------------------------------------------- packed varlen
+
+
+def _varlen_call(L, cq, ck, uq=None, uk=None, Tq=64, Tk=80, Hq=2, Hkv=2, D=64, scale=0.125,
+                 out_ptr=None, nseg=None):
+    q = _t(Tq, 0, Hq * D, D, FAKE)
+    k = _t(Tk, 0, Hkv * D, D, FAKE + (1 << 24))
+    v = _t(Tk, 0, Hkv * D, D, FAKE + (2 << 24))
+    out = _t(Tq, 0, Hq * D, D, FAKE + (3 << 24) if out_ptr is None else out_ptr)
+    n = len(cq) - 1 if nseg is None else nseg
+    arr = lambda a: ctypes.cast((ctypes.c_int32 * len(a))(*a), ctypes.c_void_p) if a is not None else None
+    return L.attn_fwd_varlen(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), arr(cq), arr(ck), arr(uq),
+                             arr(uk), n, Hq, Hkv, scale, ctypes.byref(out), D, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(cq=[0, 40, 30], ck=[0, 40, 80]),                     # cu_q decreases
+    dict(cq=[0, 30, 64], ck=[0, 50, 81]),                     # cu_k past k.len_s
+    dict(cq=[0, 30, 65], ck=[0, 50, 80]),                     # cu_q past q.len_s
+    dict(cq=[-1, 30, 64], ck=[0, 50, 80]),                    # negative start
+    dict(cq=[0, 30, 64], ck=[0, 50, 80], uq=[31, 34]),        # seqused_q > segment
+    dict(cq=[0, 30, 64], ck=[0, 50, 80], uk=[50, 31]),        # seqused_k > segment
+    dict(cq=[0, 30, 64], ck=[0, 50, 80], uk=[-1, 3]),
+    dict(cq=[0, 30, 64], ck=[0, 50, 80], scale=-1.0),
+    dict(cq=[0, 30, 64], ck=[0, 50, 80], Hq=3, Hkv=2),
+    dict(cq=[0, 30, 64], ck=[0, 50, 80], out_ptr=FAKE + 4096),  # out overlaps q
+    dict(cq=[0, 64], ck=[0, 80], nseg=-1),
+])
+def test_varlen_rejects_bad_arguments(L, kw):
+    st = _varlen_call(L, **kw)
+    assert st == INVALID, (st, L.sk_last_error())
+    assert L.sk_last_error()
+
+
+def test_varlen_rejects_unsupported_head_dim(L):
+    assert _varlen_call(L, [0, 64], [0, 80], D=96) == UNSUPPORTED
+
+
+def test_varlen_null_cu_arrays_rejected(L):
+    q = _t(64, 0, 128, 64, FAKE)
+    k = _t(80, 0, 128, 64, FAKE + (1 << 24))
+    out = _t(64, 0, 128, 64, FAKE + (3 << 24))
+    st = L.attn_fwd_varlen(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), None, None, None, None, 2, 2, 2,
+                           0.125, ctypes.byref(out), 64, None)
+    assert st == INVALID

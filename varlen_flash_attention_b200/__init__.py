@@ -9,6 +9,8 @@ rejected, ``SplitKVError`` is raised.
 Entry points (same names as the C ABI):
   attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix, real_len=None,
                     softmax_scale=None, out=None, q_valid=None)
+  attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, seqused_q=None, seqused_k=None,
+                  softmax_scale=None, out=None)
   qk_rmsnorm_rope(q, k, w_q, w_k, rope_table, rot_dim=None, interleaved=False, eps=1e-6)
   sk_device_status(device=None, clear=True), sk_set_wait_timeout_ms(ms), sk_abi_version()
 """
@@ -24,6 +26,7 @@ __all__ = [
     "SkTensor",
     "lib",
     "attn_fwd_split_kv",
+    "attn_fwd_varlen",
     "qk_rmsnorm_rope",
     "sk_device_status",
     "sk_set_wait_timeout_ms",
@@ -77,6 +80,8 @@ def lib() -> ctypes.CDLL:
             L.attn_fwd_split_kv_ex.argtypes = [P, P, P, P, P, vp, i32, i32, ctypes.c_float, P, i32, i32,
                                                vp, vp]
             L.attn_fwd_split_kv_ex.restype = i32
+            L.attn_fwd_varlen.argtypes = [P, P, P, vp, vp, vp, vp, i32, i32, i32, ctypes.c_float, P, i32, vp]
+            L.attn_fwd_varlen.restype = i32
             L.qk_rmsnorm_rope.argtypes = [P, P, vp, vp, vp, i32, i32, i32, ctypes.c_float, i32, i32,
                                           i32, i32, vp]
             L.qk_rmsnorm_rope.restype = i32
@@ -161,6 +166,49 @@ def attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix,
         st = L.attn_fwd_split_kv(*args, _stream_ptr(stream))
     else:
         st = L.attn_fwd_split_kv_ex(*args, ctypes.cast(qv, ctypes.c_void_p), _stream_ptr(stream))
+    _check(st)
+    return out
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int],
+                    seqused_q: Optional[Sequence[int]] = None,
+                    seqused_k: Optional[Sequence[int]] = None,
+                    softmax_scale: Optional[float] = None, out=None, stream=None):
+    """Packed variable-length attention: segment i's query rows
+    [cu_q[i], cu_q[i+1]) attend only to key rows [cu_k[i], cu_k[i+1]).
+
+    q [Tq, Hq, D] or [1, Tq, Hq, D]; k, v [Tk, Hkv, D] or [1, Tk, Hkv, D]
+    (bf16 CUDA, head_dim contiguous).  cu_seqlens_*: host sequences of
+    num_segments + 1 ints (computed once when the batch is packed, no device
+    sync).  seqused_*: optional host sequences of valid rows per segment (the
+    rest is pad).  Returns ``out`` shaped like ``q`` (allocated if not given;
+    rows outside every segment are left as they were).
+    """
+    import torch
+
+    def as4(t):
+        return t.unsqueeze(0) if t.dim() == 3 else t
+
+    q4, k4, v4 = as4(q), as4(k), as4(v)
+    if q4.shape[0] != 1 or k4.shape[0] != 1 or v4.shape[0] != 1:
+        raise ValueError("packed tensors have a single batch row")
+    _, Tq, Hq, D = q4.shape
+    Hkv = k4.shape[2]
+    if out is None:
+        out = torch.zeros_like(q)
+    o4 = as4(out)
+    if softmax_scale is None:
+        softmax_scale = D ** -0.5
+    n = len(cu_seqlens_q) - 1
+    if n < 0 or len(cu_seqlens_k) != n + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k need num_segments + 1 entries each")
+    cq, ck = _int32_array(cu_seqlens_q, n + 1), _int32_array(cu_seqlens_k, n + 1)
+    uq, uk = _int32_array(seqused_q, n), _int32_array(seqused_k, n)
+    descs = [tensor_desc(t) for t in (q4, k4, v4, o4)]
+    cp = lambda a: ctypes.cast(a, ctypes.c_void_p) if a is not None else None
+    st = lib().attn_fwd_varlen(ctypes.byref(descs[0]), ctypes.byref(descs[1]), ctypes.byref(descs[2]),
+                               cp(cq), cp(ck), cp(uq), cp(uk), n, Hq, Hkv, float(softmax_scale),
+                               ctypes.byref(descs[3]), D, _stream_ptr(stream))
     _check(st)
     return out
 

@@ -1,7 +1,8 @@
 // Split-KV tail-padded attention forward for sm_100a.
 //
 // One CTA computes two 128-row query tiles (A and B, 256 consecutive rows) of
-// one (batch row, query head):
+// one (entry, query head), an entry being a batch row or, for packed varlen
+// input, one segment:
 //   O = softmax(scale * Q K*^T) V*,  K*/V* = cat(prefix, suffix)[0:real_len]
 // ("sglang PR 26973", forward_with_replicated_kv_prefix; "sglang PR 30107",
 // tail_attn_meta / tail-pad layout invariant).  The concatenation is never
@@ -103,9 +104,10 @@ struct alignas(64) AttnParams {
   int32_t q_valid[kMaxBatch];   // query rows that are real
   int32_t n_prefix[kMaxBatch];  // valid prefix keys = min(Sp, real_len)
   int32_t n_suffix[kMaxBatch];  // valid suffix keys = max(0, real_len - Sp)
-  uint16_t* out;                // element (b0, 0, 0, 0) of this launch's first batch row
-  int64_t out_sb, out_ss, out_sh;
-  int32_t Sq;
+  int32_t sq[kMaxBatch];        // output rows of the entry (rows in [q_valid, sq) are written as zeros)
+  int64_t out_off[kMaxBatch];   // element offset of the entry's row 0, head 0 from `out`
+  uint16_t* out;
+  int64_t out_ss, out_sh;
   int32_t group;                // num_q_heads / num_kv_heads
   float scale_log2;             // softmax_scale * log2(e)
   int32_t* status;              // device status word
@@ -318,11 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const int tP = (nkp + kBlockN - 1) / kBlockN;
   const int tS = (nks + kBlockN - 1) / kBlockN;
   const int n_tiles = tP + tS;
-  uint16_t* out_bh = p.out + static_cast<int64_t>(bl) * p.out_sb + static_cast<int64_t>(hq) * p.out_sh;
+  const int sq = p.sq[bl];
+  uint16_t* out_bh = p.out + p.out_off[bl] + static_cast<int64_t>(hq) * p.out_sh;
 
   if (row0 >= qv || n_tiles == 0) {
     // Every row of this CTA is pad, or this batch row has no valid key: exact zeros.
-    const int r_end = min(row0 + kRowsPerCta, p.Sq);
+    const int r_end = min(row0 + kRowsPerCta, sq);
     store_zero_rows(out_bh, p.out_ss, row0, r_end, D, threadIdx.x, kThreads);
     return;
   }
@@ -644,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         skptx::tmem_ld32(tO + c * 32, o);
         skptx::tmem_wait_ld();
         skptx::reg_fence(o);
-        if (row < p.Sq) {
+        if (row < sq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
           if (row < qv) {
 #pragma unroll

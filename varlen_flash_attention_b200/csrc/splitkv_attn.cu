@@ -254,6 +254,8 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
       prm.q_valid[i] = static_cast<int32_t>(qv);
       prm.n_prefix[i] = static_cast<int32_t>(npre);
       prm.n_suffix[i] = static_cast<int32_t>(nsuf);
+      prm.sq[i] = Sq;
+      prm.out_off[i] = static_cast<int64_t>(i) * out->stride_b;
       auto bptr = [&](const sk_tensor_t* t) {
         return static_cast<const void*>(static_cast<const uint16_t*>(t->ptr) + static_cast<int64_t>(b) * t->stride_b);
       };
@@ -269,14 +271,106 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
       }
     }
     prm.out = static_cast<uint16_t*>(out->ptr) + static_cast<int64_t>(b0) * out->stride_b;
-    prm.out_sb = out->stride_b;
     prm.out_ss = out->stride_s;
     prm.out_sh = out->stride_h;
-    prm.Sq = Sq;
     prm.group = Hq / Hkv;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.status = info->status;
     prm.wait_limit_ns = g_wait_limit_ns;
+    st = (D == 64) ? launch_attn<64>(prm, n_qtiles, Hq, nb, stream, info)
+                   : launch_attn<128>(prm, n_qtiles, Hq, nb, stream, info);
+    if (st != SK_OK) return st;
+  }
+  return SK_OK;
+}
+
+// Packed varlen input: segment i owns query rows [cu_q[i], cu_q[i+1]) and key
+// rows [cu_k[i], cu_k[i+1]) of single-row tensors; each segment becomes one
+// kernel entry whose tensor maps start at the segment's first row (no prefix,
+// the segment's keys are the suffix), so the block-diagonal mask costs nothing.
+sk_status_t varlen_impl(const sk_tensor_t* q, const sk_tensor_t* k, const sk_tensor_t* v,
+                        const int32_t* cu_q, const int32_t* cu_k, const int32_t* used_q,
+                        const int32_t* used_k, int32_t nseg, int32_t Hq, int32_t Hkv, float scale,
+                        const sk_tensor_t* out, int32_t D, void* stream_v) {
+  if (nseg < 0) return fail(SK_ERR_INVALID_ARG, "num_segments < 0");
+  if (nseg > 0 && (!cu_q || !cu_k)) return fail(SK_ERR_INVALID_ARG, "cu_seqlens arrays are NULL");
+  if (Hq <= 0 || Hkv <= 0) return fail(SK_ERR_INVALID_ARG, "head counts must be positive");
+  if (Hq % Hkv != 0) return fail(SK_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
+  if (Hq > 65535) return fail(SK_ERR_UNSUPPORTED, "num_q_heads > 65535");
+  if (D != 64 && D != 128) return fail(SK_ERR_UNSUPPORTED, "head_dim %d not in {64, 128}", D);
+  if (!(std::isfinite(scale) && scale >= 0.f)) return fail(SK_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  sk_status_t st;
+  if ((st = check_tensor("q", q, 1, Hq, D)) != SK_OK) return st;
+  if ((st = check_tensor("k", k, 1, Hkv, D)) != SK_OK) return st;
+  if ((st = check_tensor("v", v, 1, Hkv, D)) != SK_OK) return st;
+  if ((st = check_tensor("out", out, 1, Hq, D)) != SK_OK) return st;
+  if (out->len_s != q->len_s) return fail(SK_ERR_INVALID_ARG, "out.len_s (%d) != q.len_s (%d)", out->len_s, q->len_s);
+  if (k->len_s != v->len_s) return fail(SK_ERR_INVALID_ARG, "k.len_s != v.len_s");
+  if (!no_self_overlap(*out, 1, Hq, D)) return fail(SK_ERR_INVALID_ARG, "out overlaps itself");
+  if (nseg == 0) return SK_OK;
+  if (cu_q[0] < 0 || cu_k[0] < 0) return fail(SK_ERR_INVALID_ARG, "cu_seqlens[0] < 0");
+  int32_t max_sq = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int64_t lq = static_cast<int64_t>(cu_q[i + 1]) - cu_q[i];
+    const int64_t lk = static_cast<int64_t>(cu_k[i + 1]) - cu_k[i];
+    if (lq < 0 || lk < 0) return fail(SK_ERR_INVALID_ARG, "cu_seqlens decrease at segment %d", i);
+    if (used_q && (used_q[i] < 0 || used_q[i] > lq))
+      return fail(SK_ERR_INVALID_ARG, "seqused_q[%d]=%d outside [0, %lld]", i, used_q[i], (long long)lq);
+    if (used_k && (used_k[i] < 0 || used_k[i] > lk))
+      return fail(SK_ERR_INVALID_ARG, "seqused_k[%d]=%d outside [0, %lld]", i, used_k[i], (long long)lk);
+    max_sq = std::max<int32_t>(max_sq, static_cast<int32_t>(lq));
+  }
+  if (cu_q[nseg] > q->len_s) return fail(SK_ERR_INVALID_ARG, "cu_seqlens_q[%d]=%d > q.len_s=%d", nseg, cu_q[nseg], q->len_s);
+  if (cu_k[nseg] > k->len_s) return fail(SK_ERR_INVALID_ARG, "cu_seqlens_k[%d]=%d > k.len_s=%d", nseg, cu_k[nseg], k->len_s);
+  if (max_sq == 0) return SK_OK;
+  Span so, si;
+  span_of(*out, 1, Hq, D, &so);
+  const struct { const char* n; const sk_tensor_t* t; int H; } ins[3] = {{"q", q, Hq}, {"k", k, Hkv}, {"v", v, Hkv}};
+  for (auto& in : ins) {
+    span_of(*in.t, 1, in.H, D, &si);
+    if (overlaps(so, si)) return fail(SK_ERR_INVALID_ARG, "out overlaps %s", in.n);
+  }
+
+  int dev = 0;
+  DeviceInfo* info = nullptr;
+  if ((st = device_setup(&dev, &info)) != SK_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  auto rptr = [](const sk_tensor_t* t, int64_t row) {
+    return static_cast<const void*>(static_cast<const uint16_t*>(t->ptr) + row * t->stride_s);
+  };
+  for (int s0 = 0; s0 < nseg; s0 += skattn::kMaxBatch) {
+    const int nb = std::min(skattn::kMaxBatch, nseg - s0);
+    skattn::AttnParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    int32_t chunk_sq = 0;
+    for (int i = 0; i < nb; ++i) {
+      const int g = s0 + i;
+      const int32_t lq = cu_q[g + 1] - cu_q[g];
+      const int32_t lk = cu_k[g + 1] - cu_k[g];
+      const int32_t nk = used_k ? used_k[g] : lk;
+      const int32_t qv = used_q ? used_q[g] : lq;
+      prm.q_valid[i] = qv;
+      prm.n_prefix[i] = 0;
+      prm.n_suffix[i] = nk;
+      prm.sq[i] = lq;
+      prm.out_off[i] = static_cast<int64_t>(cu_q[g]) * out->stride_s;
+      chunk_sq = std::max(chunk_sq, lq);
+      if (qv > 0 && nk > 0)
+        if ((st = encode_map(&prm.tm_q[i], rptr(q, cu_q[g]), q->stride_s, q->stride_h, Hq, qv, D)) != SK_OK) return st;
+      if (nk > 0) {
+        if ((st = encode_map(&prm.tm_ks[i], rptr(k, cu_k[g]), k->stride_s, k->stride_h, Hkv, nk, D)) != SK_OK) return st;
+        if ((st = encode_map(&prm.tm_vs[i], rptr(v, cu_k[g]), v->stride_s, v->stride_h, Hkv, nk, D)) != SK_OK) return st;
+      }
+    }
+    if (chunk_sq == 0) continue;
+    prm.out = static_cast<uint16_t*>(out->ptr);
+    prm.out_ss = out->stride_s;
+    prm.out_sh = out->stride_h;
+    prm.group = Hq / Hkv;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.status = info->status;
+    prm.wait_limit_ns = g_wait_limit_ns;
+    const int n_qtiles = (chunk_sq + skattn::kRowsPerCta - 1) / skattn::kRowsPerCta;
     st = (D == 64) ? launch_attn<64>(prm, n_qtiles, Hq, nb, stream, info)
                    : launch_attn<128>(prm, n_qtiles, Hq, nb, stream, info);
     if (st != SK_OK) return st;
@@ -309,6 +403,19 @@ sk_status_t attn_fwd_split_kv_ex(const sk_tensor_t* q, const sk_tensor_t* k_pref
   try {
     return attn_impl(q, k_prefix, v_prefix, k_suffix, v_suffix, real_len, num_q_heads, num_kv_heads,
                      softmax_scale, out, batch, head_dim, q_valid, stream);
+  } catch (...) {
+    return fail(SK_ERR_INVALID_ARG, "internal exception");
+  }
+}
+
+sk_status_t attn_fwd_varlen(const sk_tensor_t* q, const sk_tensor_t* k, const sk_tensor_t* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            const int32_t* seqused_q, const int32_t* seqused_k, int32_t num_segments,
+                            int32_t num_q_heads, int32_t num_kv_heads, float softmax_scale,
+                            const sk_tensor_t* out, int32_t head_dim, void* stream) {
+  try {
+    return varlen_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, seqused_q, seqused_k, num_segments,
+                       num_q_heads, num_kv_heads, softmax_scale, out, head_dim, stream);
   } catch (...) {
     return fail(SK_ERR_INVALID_ARG, "internal exception");
   }
