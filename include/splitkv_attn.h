@@ -187,6 +187,17 @@ SK_API sk_status_t sk_device_status(int32_t device, int32_t* status_out, int32_t
 /* Bound on every in-kernel wait, in milliseconds (default 2000; 1..60000). */
 SK_API sk_status_t sk_set_wait_timeout_ms(int32_t ms);
 
+/*
+ * sk_test_stall_mma — test hook for the failure path (no counterpart on the
+ * pages).  While on != 0, the attention kernels' MMA warp first waits on a
+ * barrier that nothing arrives at, so every in-kernel wait runs out after the
+ * sk_set_wait_timeout_ms limit: each CTA raises SK_ERR_DEVICE_TIMEOUT in the
+ * device status word, drains its own copies, frees TMEM and exits, and the
+ * context stays usable.  Outputs of such calls are undefined.  Off by default;
+ * returns SK_OK.
+ */
+SK_API sk_status_t sk_test_stall_mma(int32_t on);
+
 /* ABI version of this header (increments on incompatible change). */
 SK_API int32_t sk_abi_version(void);
 

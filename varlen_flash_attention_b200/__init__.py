@@ -30,6 +30,7 @@ __all__ = [
     "qk_rmsnorm_rope",
     "sk_device_status",
     "sk_set_wait_timeout_ms",
+    "sk_test_stall_mma",
     "sk_abi_version",
     "tensor_desc",
     "LIB_PATH",
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
             L.sk_device_status.restype = i32
             L.sk_set_wait_timeout_ms.argtypes = [i32]
             L.sk_set_wait_timeout_ms.restype = i32
+            L.sk_test_stall_mma.argtypes = [i32]
+            L.sk_test_stall_mma.restype = i32
             L.sk_abi_version.argtypes = []
             L.sk_abi_version.restype = i32
             _lib = L
@@ -252,6 +255,11 @@ def sk_device_status(device: Optional[int] = None, clear: bool = True) -> int:
 
 def sk_set_wait_timeout_ms(ms: int) -> None:
     _check(lib().sk_set_wait_timeout_ms(int(ms)))
+
+
+def sk_test_stall_mma(on: bool) -> None:
+    """Test hook: make every in-kernel wait run out (see include/splitkv_attn.h)."""
+    _check(lib().sk_test_stall_mma(int(bool(on))))
 
 
 def sk_abi_version() -> int:

@@ -112,6 +112,7 @@ struct alignas(64) AttnParams {
   float scale_log2;             // softmax_scale * log2(e)
   int32_t* status;              // device status word
   uint64_t wait_limit_ns;
+  int32_t test_stall;           // test hook: the MMA warp first waits on a barrier nothing arrives at
 };
 
 template <int D>
@@ -434,6 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint64_t dV = skptx::sdesc_sw128(sbase + L::kV, L::kSub, 1024);
     const uint64_t dP = skptx::sdesc_sw128(sbase + L::kP, 16, 1024);
     bool ok = W.wait_warp(bar(L::bQFull), 0) && W.wait_warp(bar(L::bKFull), 0);
+    // Test hook for the bounded-wait path: MmaDone is only committed by this
+    // warp after its loop, so this wait runs out (every role then aborts,
+    // drains and exits with SK_ERR_DEVICE_TIMEOUT in the status word).
+    if (p.test_stall) ok = ok && W.wait_warp(bar(L::bMmaDone), 0);
 #if SKA_TRACE
     if (lane == 0) SKA_TR(0, 1, 0);
 #endif

@@ -45,6 +45,7 @@ sk_status_t cuda_fail(cudaError_t e, const char* what) {
 __device__ int32_t g_device_status = 0;
 
 uint64_t g_wait_limit_ns = 2000ull * 1000ull * 1000ull;
+int32_t g_test_stall = 0;
 std::mutex g_mu;
 
 struct DeviceInfo {
@@ -277,6 +278,7 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.status = info->status;
     prm.wait_limit_ns = g_wait_limit_ns;
+    prm.test_stall = g_test_stall;
     st = (D == 64) ? launch_attn<64>(prm, n_qtiles, Hq, nb, stream, info)
                    : launch_attn<128>(prm, n_qtiles, Hq, nb, stream, info);
     if (st != SK_OK) return st;
@@ -370,6 +372,7 @@ sk_status_t varlen_impl(const sk_tensor_t* q, const sk_tensor_t* k, const sk_ten
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.status = info->status;
     prm.wait_limit_ns = g_wait_limit_ns;
+    prm.test_stall = g_test_stall;
     const int n_qtiles = (chunk_sq + skattn::kRowsPerCta - 1) / skattn::kRowsPerCta;
     st = (D == 64) ? launch_attn<64>(prm, n_qtiles, Hq, nb, stream, info)
                    : launch_attn<128>(prm, n_qtiles, Hq, nb, stream, info);
@@ -511,6 +514,12 @@ sk_status_t sk_set_wait_timeout_ms(int32_t ms) {
   if (ms < 1 || ms > 60000) return fail(SK_ERR_INVALID_ARG, "timeout must be in [1, 60000] ms");
   std::lock_guard<std::mutex> lk(g_mu);
   g_wait_limit_ns = static_cast<uint64_t>(ms) * 1000000ull;
+  return SK_OK;
+}
+
+sk_status_t sk_test_stall_mma(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_test_stall = on ? 1 : 0;
   return SK_OK;
 }
 
