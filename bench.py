@@ -65,13 +65,21 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def measured_peaks():
+SUSTAINED_AFTER_S = 1.0  # a timed region longer than this runs under the power cap
+
+
+def measured_peaks(timed_s: float = 0.0):
+    """(peak TFLOP/s, description): the measured cuBLAS bf16 burst figure for a
+    kernel timed briefly, the sustained (power-capped) one for a timed region
+    longer than SUSTAINED_AFTER_S; the recipe's fallback if no measurement."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["bf16_tflops"]), "measured"
-    return FALLBACK_BF16_TFLOPS, "fallback"
+        if timed_s > SUSTAINED_AFTER_S and "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"]), "measured bf16 sustained"
+        return float(d["bf16_tflops"]), "measured bf16 burst"
+    return FALLBACK_BF16_TFLOPS, "fallback bf16 burst"
 
 
 def traffic_per_launch(workload):
@@ -334,7 +342,7 @@ def run_ours(args, w):
     barrier(dist)
     _, e2e_value = combine_ranks(fl, args.steps, ev0.elapsed_time(ev1), dist)
 
-    peak, peak_kind = measured_peaks()
+    peak, peak_kind = measured_peaks(dt_ms_max / 1e3)
     clocks = clk.summary()
     line = None
     if rank == 0:
@@ -357,7 +365,7 @@ def run_ours(args, w):
                        "flop_per_step": fl, "l2": "inputs rotate over 4 device copies (> 126 MB L2)",
                        "parallelism": f"replica x{world}" if world > 1 else "single"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "peak_kind": f"{peak_kind} bf16 burst",
+                         "frac": achieved / peak, "peak_kind": peak_kind,
                          "traffic": traffic_per_launch(w.name)},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,

@@ -65,3 +65,21 @@ def test_flops_count_only_valid_rows_and_keys():
     assert bench.flops_of(w) == 4.0 * 128 * 32 * 25048 * 25048
     w = workloads.get("cross_short_kv")
     assert bench.flops_of(w) == 4.0 * 128 * 16 * 32760 * 1024
+
+
+def test_peak_choice_burst_vs_sustained():
+    import json
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+
+    peaks = os.path.join(bench.ROOT, "MEASURED_PEAKS.json")
+    if not os.path.exists(peaks):
+        pytest.skip("no measured peaks on this machine")
+    d = json.load(open(peaks))
+    p_short, k_short = bench.measured_peaks(0.05)
+    p_long, k_long = bench.measured_peaks(5.0)
+    assert p_short == d["bf16_tflops"] and "burst" in k_short
+    if "bf16_tflops_sustained" in d:
+        assert p_long == d["bf16_tflops_sustained"] and "sustained" in k_long
