@@ -315,32 +315,60 @@ def run_ours(args, w):
     per_launch_ms = dt_ms / args.steps
     achieved = fl / (per_launch_ms / 1e3) / 1e12
 
-    # ---- end to end through the public API with host buffers (pinned), H2D + kernel + D2H
+    # ---- end to end through the public API with host buffers (pinned): every
+    # step copies its inputs host -> device, runs the kernel and reads its
+    # output back.  Three streams pipeline consecutive steps (step i+1's
+    # inputs upload while step i computes and step i-1's output downloads),
+    # with two device buffer sets and two pinned output buffers.
     pinned = {k: host[k].pin_memory() for k in keys}
-    out_host = torch.empty(w.B, w.Sq, w.Hq, w.D, dtype=torch.bfloat16).pin_memory()
+    outs_host = [torch.empty(w.B, w.Sq, w.Hq, w.D, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     h2d = sum(pinned[k].numel() * 2 for k in keys)
-    d2h = out_host.numel() * 2
-    dbuf = {k: torch.empty_like(copies[0][k]) for k in keys}
-    dout = torch.empty_like(outs[0])
+    d2h = outs_host[0].numel() * 2
+    dbufs = [{k: torch.empty_like(copies[0][k]) for k in keys} for _ in range(2)]
+    douts = [torch.empty_like(outs[0]) for _ in range(2)]
+    s_up, s_run, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_run = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
+    primed = [False, False]
 
-    def e2e_step():
-        for k in keys:
-            dbuf[k].copy_(pinned[k], non_blocking=True)
-        sk.attn_fwd_split_kv(dbuf["q"], dbuf["k_prefix"], dbuf["v_prefix"], dbuf["k_suffix"],
-                             dbuf["v_suffix"], real_len=rl, out=dout, stream=stream)
-        out_host.copy_(dout, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(s_up):
+            if primed[b]:
+                s_up.wait_event(ev_run[b])  # the kernel of step i-2 has read this buffer set
+            for k in keys:
+                dbufs[b][k].copy_(pinned[k], non_blocking=True)
+            ev_up[b].record(s_up)
+        s_run.wait_event(ev_up[b])
+        if primed[b]:
+            s_run.wait_event(ev_down[b])    # step i-2's output has been read back
+        sk.attn_fwd_split_kv(dbufs[b]["q"], dbufs[b]["k_prefix"], dbufs[b]["v_prefix"], dbufs[b]["k_suffix"],
+                             dbufs[b]["v_suffix"], real_len=rl, out=douts[b], stream=s_run)
+        ev_run[b].record(s_run)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev_run[b])
+            outs_host[b].copy_(douts[b], non_blocking=True)
+            ev_down[b].record(s_down)
+        primed[b] = True
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    for i in range(max(2, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier(dist)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    ev1.record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_up)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(s_down)  # the d2h stream ends after every step's read-back
     torch.cuda.synchronize(dev)
     barrier(dist)
-    _, e2e_value = combine_ranks(fl, args.steps, ev0.elapsed_time(ev1), dist)
+    _, e2e_value = combine_ranks(fl, args.steps, e0.elapsed_time(e1), dist)
+    if sk.sk_device_status(local, clear=True) != 0:
+        raise RuntimeError("device status set during the end-to-end run")
+    # same inputs, deterministic kernel: the last read-back equals the device-timed output
+    if not torch.equal(outs_host[(args.steps - 1) % 2].view(torch.int16), outs[0].cpu().view(torch.int16)):
+        raise RuntimeError("end-to-end output differs from the device-timed output")
 
     peak, peak_kind = measured_peaks(dt_ms_max / 1e3)
     clocks = clk.summary()
