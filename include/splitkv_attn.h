@@ -173,6 +173,27 @@ SK_API sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, c
                             int32_t num_q_heads, int32_t num_kv_heads, int32_t batch,
                             int32_t head_dim, void* stream);
 
+/*
+ * sk_shard_pad_copy — one rank's chunk of a tail-padded sequence shard
+ * ("sglang PR 30107", shard_like: pad the tail of the stream with num_pad rows
+ * of zeros or repeats of its last row, then take rows [first_row,
+ * first_row + dst_rows)), in one pass that reads only the chunk's real rows.
+ * Needed only on the rank whose chunk holds pad; other chunks are views.
+ *
+ *   src   device, rows of row_bytes bytes: row s of batch b at
+ *         src + b*src_stride_b + s*src_stride_s, s < src_rows (read)
+ *   dst   device, dst_rows rows per batch row at dst + b*dst_stride_b +
+ *         r*dst_stride_s (written); must not overlap src or itself
+ *   row   r of dst = src row first_row + r if < src_rows, else zeros
+ *         (pad_mode 0) or src row src_rows - 1 (pad_mode 1)
+ *   row_bytes and all strides multiples of 16, pointers 16-byte aligned.
+ * Returns SK_OK, SK_ERR_INVALID_ARG or SK_ERR_CUDA; launches on `stream`.
+ */
+SK_API sk_status_t sk_shard_pad_copy(const void* src, int64_t src_stride_b, int64_t src_stride_s,
+                                     int32_t src_rows, void* dst, int64_t dst_stride_b,
+                                     int64_t dst_stride_s, int32_t dst_rows, int32_t first_row,
+                                     int32_t row_bytes, int32_t batch, int32_t pad_mode, void* stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if none). */
 SK_API const char* sk_last_error(void);
 

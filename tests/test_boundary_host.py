@@ -210,3 +210,27 @@ def test_varlen_null_cu_arrays_rejected(L):
     st = L.attn_fwd_varlen(ctypes.byref(q), ctypes.byref(k), ctypes.byref(k), None, None, None, None, 2, 2, 2,
                            0.125, ctypes.byref(out), 64, None)
     assert st == INVALID
+
+
+# ---------------------------------------------------------------- shard pad copy
+
+
+@pytest.mark.parametrize("kw", [
+    dict(row_bytes=24),                   # not a multiple of 16
+    dict(row_bytes=0),
+    dict(src_ss=100),                     # stride not a multiple of 16
+    dict(pad_mode=2),
+    dict(dst_rows=-1),
+    dict(src_rows=0, pad_mode=1),         # repeat_last without a source row
+    dict(dst=FAKE + 8),                   # misaligned
+    dict(dst=FAKE + 64),                  # overlaps src
+    dict(dst_ss=16, row_bytes=32),        # destination rows overlap
+])
+def test_shard_pad_copy_rejects_bad_arguments(L, kw):
+    a = dict(src=FAKE, src_sb=1 << 20, src_ss=256, src_rows=100, dst=FAKE + (1 << 24), dst_sb=1 << 16,
+             dst_ss=256, dst_rows=13, first_row=91, row_bytes=256, batch=2, pad_mode=0)
+    a.update(kw)
+    st = L.sk_shard_pad_copy(a["src"], a["src_sb"], a["src_ss"], a["src_rows"], a["dst"], a["dst_sb"],
+                             a["dst_ss"], a["dst_rows"], a["first_row"], a["row_bytes"], a["batch"],
+                             a["pad_mode"], None)
+    assert st == INVALID, (st, L.sk_last_error())

@@ -174,3 +174,25 @@ def test_gather_inverts_shard_on_gloo_ranks(world, S):
     for rank, size, r, lp, ok in res:
         assert size == world and r == rank and ok
         assert lp == (num_pad if rank == world - 1 else 0)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("S, sp, mode", [(4429, 8, "zeros"), (10, 4, "repeat_last"), (1, 4, "zeros"),
+                                          (1, 4, "repeat_last"), (333, 16, "zeros")])
+def test_shard_copy_kernel_matches_torch(S, sp, mode):
+    """The CUDA one-pass copy (chunks holding pad) equals the torch path bitwise."""
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from varlen_flash_attention_b200 import build
+
+    build.build()
+    g = torch.Generator().manual_seed(S)
+    x = torch.randn(2, S, 3, 64, generator=g).to(torch.bfloat16)
+    xd = x.cuda()
+    for r in range(sp):
+        p = sps.build_shard_plan(S, sp_size=sp, sp_rank=r)
+        ref = sps.shard_like(x, p, pad_mode=mode)          # CPU: torch ops
+        got = sps.shard_like(xd, p, pad_mode=mode)         # CUDA: view or the copy kernel
+        torch.cuda.synchronize()
+        assert got.shape == ref.shape
+        assert torch.equal(got.cpu().view(torch.int16), ref.view(torch.int16)), f"rank {r}"

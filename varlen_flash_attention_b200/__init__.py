@@ -27,6 +27,7 @@ __all__ = [
     "lib",
     "attn_fwd_split_kv",
     "attn_fwd_varlen",
+    "sk_shard_pad_copy",
     "qk_rmsnorm_rope",
     "sk_device_status",
     "sk_set_wait_timeout_ms",
@@ -81,6 +82,9 @@ def lib() -> ctypes.CDLL:
             L.attn_fwd_split_kv_ex.argtypes = [P, P, P, P, P, vp, i32, i32, ctypes.c_float, P, i32, i32,
                                                vp, vp]
             L.attn_fwd_split_kv_ex.restype = i32
+            i64 = ctypes.c_int64
+            L.sk_shard_pad_copy.argtypes = [vp, i64, i64, i32, vp, i64, i64, i32, i32, i32, i32, i32, vp]
+            L.sk_shard_pad_copy.restype = i32
             L.attn_fwd_varlen.argtypes = [P, P, P, vp, vp, vp, vp, i32, i32, i32, ctypes.c_float, P, i32, vp]
             L.attn_fwd_varlen.restype = i32
             L.qk_rmsnorm_rope.argtypes = [P, P, vp, vp, vp, i32, i32, i32, ctypes.c_float, i32, i32,
@@ -214,6 +218,30 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence
                                ctypes.byref(descs[3]), D, _stream_ptr(stream))
     _check(st)
     return out
+
+
+def sk_shard_pad_copy(src, dst, first_row: int, pad_mode: str = "zeros", stream=None):
+    """dst[:, r] = src[:, first_row + r] while that row exists, else zeros
+    (``pad_mode="zeros"``) or src's last row (``"repeat_last"``): one rank's
+    chunk of a tail-padded shard in one pass.  src [B, S, ...], dst
+    [B, L, ...] CUDA tensors of one dtype with contiguous rows (dims >= 2)."""
+    if src.dtype != dst.dtype or src.shape[0] != dst.shape[0] or src.shape[2:] != dst.shape[2:]:
+        raise ValueError("src and dst must share dtype, batch and row shape")
+    row_elems = 1
+    for d in src.shape[2:]:
+        row_elems *= d
+    es = src.element_size()
+    for t in (src, dst):
+        if t.numel() and (not t.is_cuda or t[:1, :1].reshape(-1).numel() != row_elems or
+                          not t[0, 0].is_contiguous()):
+            raise ValueError("expected CUDA tensors with contiguous rows")
+    mode = {"zeros": 0, "repeat_last": 1}[pad_mode]
+    st = lib().sk_shard_pad_copy(src.data_ptr() if src.numel() else None, src.stride(0) * es, src.stride(1) * es,
+                                 src.shape[1], dst.data_ptr(), dst.stride(0) * es, dst.stride(1) * es,
+                                 dst.shape[1], int(first_row), row_elems * es, src.shape[0], mode,
+                                 _stream_ptr(stream))
+    _check(st)
+    return dst
 
 
 def qk_rmsnorm_rope(q, k, w_q, w_k, rope_table, rot_dim: Optional[int] = None,

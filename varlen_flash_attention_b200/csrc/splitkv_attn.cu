@@ -18,6 +18,7 @@
 #include "../../include/splitkv_attn.h"
 #include "attn_fwd_sm100.cuh"
 #include "qk_norm_rope.cuh"
+#include "shard_copy.cuh"
 
 namespace {
 
@@ -51,6 +52,7 @@ std::mutex g_mu;
 struct DeviceInfo {
   bool checked = false;
   bool sm100 = false;
+  int sm_count = 0;
   int32_t* status = nullptr;
   bool attn_attr_set[2] = {false, false};
 };
@@ -71,6 +73,8 @@ sk_status_t device_setup(int* dev_out, DeviceInfo** info_out) {
     e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     d.sm100 = (major == 10 && minor == 0);
+    e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_device_status);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
@@ -419,6 +423,62 @@ sk_status_t attn_fwd_varlen(const sk_tensor_t* q, const sk_tensor_t* k, const sk
   try {
     return varlen_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, seqused_q, seqused_k, num_segments,
                        num_q_heads, num_kv_heads, softmax_scale, out, head_dim, stream);
+  } catch (...) {
+    return fail(SK_ERR_INVALID_ARG, "internal exception");
+  }
+}
+
+sk_status_t sk_shard_pad_copy(const void* src, int64_t src_stride_b, int64_t src_stride_s, int32_t src_rows,
+                              void* dst, int64_t dst_stride_b, int64_t dst_stride_s, int32_t dst_rows,
+                              int32_t first_row, int32_t row_bytes, int32_t batch, int32_t pad_mode,
+                              void* stream) {
+  try {
+    if (batch < 0 || src_rows < 0 || dst_rows < 0 || first_row < 0)
+      return fail(SK_ERR_INVALID_ARG, "negative size");
+    if (row_bytes <= 0 || row_bytes % 16 != 0) return fail(SK_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 16");
+    if (pad_mode != 0 && pad_mode != 1) return fail(SK_ERR_INVALID_ARG, "pad_mode must be 0 (zeros) or 1 (repeat last)");
+    if (pad_mode == 1 && src_rows == 0 && dst_rows > 0) return fail(SK_ERR_INVALID_ARG, "repeat_last needs a source row");
+    if (batch == 0 || dst_rows == 0) return SK_OK;
+    const int64_t st[4] = {src_stride_b, src_stride_s, dst_stride_b, dst_stride_s};
+    for (int64_t v : st)
+      if (v < 0 || v % 16 != 0) return fail(SK_ERR_INVALID_ARG, "strides must be non-negative multiples of 16 bytes");
+    if (!dst || (src_rows > 0 && !src)) return fail(SK_ERR_INVALID_ARG, "NULL pointer");
+    if (reinterpret_cast<uintptr_t>(dst) % 16 || reinterpret_cast<uintptr_t>(src) % 16)
+      return fail(SK_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    if (dst_stride_s < row_bytes) return fail(SK_ERR_INVALID_ARG, "dst rows overlap");
+    if (batch > 1 && dst_stride_b < static_cast<int64_t>(dst_rows) * dst_stride_s)
+      return fail(SK_ERR_INVALID_ARG, "dst batch rows overlap");
+    // destination must not overlap the source rows it reads
+    if (src_rows > 0) {
+      const uintptr_t d0 = reinterpret_cast<uintptr_t>(dst);
+      const uintptr_t d1 = d0 + static_cast<uintptr_t>((batch - 1) * dst_stride_b + (dst_rows - 1) * dst_stride_s + row_bytes);
+      const uintptr_t s0 = reinterpret_cast<uintptr_t>(src);
+      const uintptr_t s1 = s0 + static_cast<uintptr_t>((batch - 1) * src_stride_b + (src_rows - 1) * src_stride_s + row_bytes);
+      if (d0 < s1 && s0 < d1) return fail(SK_ERR_INVALID_ARG, "dst overlaps src");
+    }
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    sk_status_t stt;
+    if ((stt = device_setup(&dev, &info)) != SK_OK) return stt;
+    skshard::PadCopyParams prm;
+    prm.src = static_cast<const uint8_t*>(src);
+    prm.dst = static_cast<uint8_t*>(dst);
+    prm.src_sb = src_stride_b;
+    prm.src_ss = src_stride_s;
+    prm.dst_sb = dst_stride_b;
+    prm.dst_ss = dst_stride_s;
+    prm.src_rows = src_rows;
+    prm.dst_rows = dst_rows;
+    prm.first_row = first_row;
+    prm.row_chunks = row_bytes / 16;
+    prm.batch = batch;
+    prm.repeat_last = pad_mode;
+    const int64_t total = static_cast<int64_t>(batch) * dst_rows * prm.row_chunks;
+    const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, int64_t(info->sm_count) * 8));
+    skshard::pad_copy_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "pad_copy_kernel launch");
+    return SK_OK;
   } catch (...) {
     return fail(SK_ERR_INVALID_ARG, "internal exception");
   }

@@ -125,24 +125,44 @@ def shard_like(x: torch.Tensor, shard: SpShard, dim: int = 1, pad_mode: str = "z
     pad the tail of ``dim`` with ``num_pad`` rows (zeros, or copies of the last
     row with ``pad_mode="repeat_last"``), then take this rank's ``local_len``
     rows.  Tensors of one stream (hidden states, RoPE tables, ...) sharded
-    with the same plan stay aligned chunk for chunk."""
+    with the same plan stay aligned chunk for chunk.
+
+    A chunk without pad is returned as a view of ``x`` (no copy).  A chunk
+    holding pad is built in one pass: on CUDA with ``dim == 1`` and
+    16-byte rows by the library's copy kernel (``sk_shard_pad_copy``), which
+    reads only the chunk's real rows; otherwise with torch ops."""
     if x.shape[dim] != shard.orig_len:
         raise ValueError(f"dim {dim} has {x.shape[dim]} rows, plan expects {shard.orig_len}")
+    if pad_mode not in ("zeros", "repeat_last"):
+        raise ValueError(f"unknown pad_mode {pad_mode!r}")
     if shard.sp_size <= 1:
         return x
-    if shard.num_pad > 0:
-        if pad_mode == "repeat_last":
-            if shard.orig_len == 0:
-                raise ValueError("repeat_last needs at least one row")
-            last = x.narrow(dim, x.shape[dim] - 1, 1)
-            x = torch.cat([x, last.expand(*[shard.num_pad if i == dim else -1 for i in range(x.dim())])], dim=dim)
-        elif pad_mode == "zeros":
-            nd = dim % x.dim()
-            pads = [0, 0] * (x.dim() - 1 - nd) + [0, shard.num_pad]
-            x = F.pad(x, pads)
-        else:
-            raise ValueError(f"unknown pad_mode {pad_mode!r}")
-    return x.narrow(dim, shard.sp_rank * shard.local_len, shard.local_len)
+    start = shard.sp_rank * shard.local_len
+    if start + shard.local_len <= shard.orig_len:
+        return x.narrow(dim, start, shard.local_len)
+    if pad_mode == "repeat_last" and shard.orig_len == 0:
+        raise ValueError("repeat_last needs at least one row")
+    nd = dim % x.dim()
+    row_bytes = x.element_size()
+    for d in x.shape[nd + 1:]:
+        row_bytes *= d
+    if x.is_cuda and nd == 1 and x.dim() >= 2 and row_bytes % 16 == 0 and x[0, 0].is_contiguous():
+        from . import sk_shard_pad_copy
+
+        shape = list(x.shape)
+        shape[1] = shard.local_len
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+        return sk_shard_pad_copy(x, out, start, pad_mode)
+    real = x.narrow(dim, min(start, shard.orig_len), max(0, shard.orig_len - start))
+    npad = shard.local_len - real.shape[dim]
+    if pad_mode == "repeat_last":
+        last = x.narrow(dim, shard.orig_len - 1, 1)
+        pad = last.expand(*[npad if i == nd else -1 for i in range(x.dim())])
+    else:
+        pad_shape = list(x.shape)
+        pad_shape[nd] = npad
+        pad = torch.zeros(pad_shape, dtype=x.dtype, device=x.device)
+    return torch.cat([real, pad], dim=dim)
 
 
 def shard_seq(x: torch.Tensor, shard: SpShard, dim: int = 1, pad_mode: str = "zeros") -> torch.Tensor:
