@@ -409,6 +409,55 @@ def run_ours(args, w):
     return 0
 
 
+def run_prologue(args, w):
+    """The optional A0 prologue (fused Q/K RMSNorm + RoPE, in place) on the
+    workload's q and k: HBM GB/s against the measured copy bandwidth.  Bytes
+    = one read and one write of every q and k element."""
+    import numpy as np
+
+    import varlen_flash_attention_b200 as sk
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator().manual_seed(w.seed)
+    S = w.Sq
+    n_copies = 2
+    qs = [torch.randn(w.B, S, w.Hq, w.D, generator=g).to(torch.bfloat16).to(dev) for _ in range(n_copies)]
+    ks = [torch.randn(w.B, S, w.Hkv, w.D, generator=g).to(torch.bfloat16).to(dev) for _ in range(n_copies)]
+    wq = torch.ones(w.D, dtype=torch.bfloat16, device=dev)
+    wk = torch.ones(w.D, dtype=torch.bfloat16, device=dev)
+    rot = w.D
+    ang = np.arange(S)[:, None] * 10000.0 ** (-np.arange(0, rot, 2) / rot)
+    table = torch.from_numpy(np.concatenate([np.cos(ang), np.sin(ang)], 1).astype(np.float32)).to(dev)
+    step = lambda i: sk.qk_rmsnorm_rope(qs[i % n_copies], ks[i % n_copies], wq, wk, table, rot_dim=rot)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        e0.record()
+        for i in range(args.steps):
+            step(i)
+        e1.record()
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    nbytes = 2 * 2 * w.B * S * (w.Hq + w.Hkv) * w.D
+    gbs = nbytes / (ms / 1e3) / 1e9
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak, kind = (json.load(open(p))["hbm_gbs"], "measured copy") if os.path.exists(p) else (6650.0, "fallback")
+    print(json.dumps({
+        "metric": "qk_rmsnorm_rope (A0 prologue) HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "bf16 in/out, fp64 arithmetic", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.B, "seq": S, "heads_q": w.Hq, "heads_kv": w.Hkv,
+                   "head_dim": w.D, "rot_dim": rot, "bytes_per_step": nbytes,
+                   "l2": f"{n_copies} rotating q/k copies"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "peak_kind": kind, "traffic": None},
+        "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -417,9 +466,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["attention", "prologue"], default="attention",
+                    help="prologue: time the optional fused Q/K RMSNorm+RoPE kernel instead")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = workloads.get(args.workload)
+    if args.op == "prologue":
+        return run_prologue(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)
