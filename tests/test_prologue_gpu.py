@@ -1,9 +1,12 @@
 """Parity of the fused Q/K RMSNorm + RoPE prologue kernel with the fp64 oracle.
 
 Bar: every output element within 1 bf16 ulp of the oracle and at least
-99.99% bit-identical.  The kernel computes in fp64 with the oracle's rounding
-points, so in practice every element is identical; the ulp allowance covers a
-sum-of-squares reduction order that differs from the oracle's sequential one.
+99.99% bit-identical on the ordinary cases, where the ulp allowance covers a
+sum-of-squares reduction order that differs from the oracle's sequential one
+(it only matters when the row's squares span more than fp64's precision).
+The special-value, multi-block and large cases demand every bit: the kernel
+decides each bf16 rounding either from an fp32 value whose error bound
+keeps it off the rounding midpoint or by recomputing the element in fp64.
 """
 import numpy as np
 import pytest
@@ -85,3 +88,103 @@ def test_prologue_in_place_on_fused_qkv_view(sk):
     ref_k = oracle.qk_rmsnorm_rope(qkv[:, :, Hq:Hq + Hkv].contiguous(), wk, tab.numpy(), eps=eps)
     _ulp_check(got[:, :, :Hq].contiguous().view(torch.int16).numpy().view(np.uint16), ref_q)
     _ulp_check(got[:, :, Hq:Hq + Hkv].contiguous().view(torch.int16).numpy().view(np.uint16), ref_k)
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _run_both(sk, q, k, wq, wk, tab, rot, inter, eps):
+    S = q.shape[1]
+    eps32 = float(np.float32(eps))
+    ref_q = oracle.qk_rmsnorm_rope(q, wq, tab.numpy(), rot_dim=rot, interleaved=inter, eps=eps32)
+    ref_k = oracle.qk_rmsnorm_rope(k, wk, tab.numpy(), rot_dim=rot, interleaved=inter, eps=eps32)
+    qd, kd = q.cuda(), k.cuda()
+    tabd = tab.cuda() if rot else torch.zeros(S, 8, device="cuda")
+    sk.qk_rmsnorm_rope(qd, kd, wq.cuda(), wk.cuda(), tabd, rot_dim=rot, interleaved=inter, eps=eps)
+    torch.cuda.synchronize()
+    return _bits(qd.cpu()), ref_q, _bits(kd.cpu()), ref_k
+
+
+@pytest.mark.parametrize("inter", [False, True])
+def test_prologue_special_values_bit_exact(sk, inter):
+    """Rows that leave the kernel's fast path (bf16 subnormals, zero rows with
+    eps = 0, inf/NaN inputs, weights and table entries near the top of the
+    range) mixed with ordinary rows: every output bit equals the oracle's."""
+    gen = torch.Generator().manual_seed(11 + int(inter))
+    B, S, Hq, Hkv, D, rot = 1, 40, 5, 3, 128, 96
+    q = torch.randn(B, S, Hq, D, generator=gen)
+    k = torch.randn(B, S, Hkv, D, generator=gen)
+    q[0, 1, 2] = 0.0                                   # zero row: r = 1/sqrt(eps)
+    q[0, 2, 0, :] *= 1e-38                             # bf16 subnormal inputs
+    q[0, 3, 1, 5] = 3e38                               # one huge value dwarfs the rest
+    q[0, 4, 4, 7] = float("inf")
+    k[0, 5, 1, 9] = float("nan")
+    k[0, 6, 2, :64] = 0.0                              # half-zero row
+    k[0, 7, 0, 3] = 1e-40                              # subnormal next to normal values
+    k[0, 3, 0, :] = -0.0                               # negative-zero row
+    q[0, 9, 1, 100:110] = -0.0                         # negative zeros past rot_dim
+    q[0, 11, 3, 10:40] = -0.0                          # negative zeros in rotated dims
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    wq = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk[17] = 1e-39                                     # y of that dim in bf16's subnormal range
+    tab = _table(S, rot)
+    tab[9, 3] = 1e38                                   # huge cos: overflowing rotation
+    tab[10, rot // 2 + 1] = -3e38
+    for eps in (1e-6, 0.0):
+        q0 = q.clone()
+        q0[0, 8, 3] = 0.0 if eps == 0.0 else q0[0, 8, 3]
+        gq, rq, gk, rk = _run_both(sk, q0, k, wq, wk, tab, rot, inter, eps)
+        assert np.array_equal(gq, rq), np.argwhere(gq != rq)[:5]
+        assert np.array_equal(gk, rk), np.argwhere(gk != rk)[:5]
+
+
+def test_prologue_huge_weight_bit_exact(sk):
+    """A weight near bf16's maximum overflows y to inf on some rows; the
+    rotation then spreads inf/NaN to the partner dims exactly as in the
+    oracle."""
+    gen = torch.Generator().manual_seed(5)
+    B, S, Hq, Hkv, D, rot = 2, 9, 4, 2, 64, 64
+    q = torch.randn(B, S, Hq, D, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, S, Hkv, D, generator=gen).to(torch.bfloat16)
+    wq = torch.ones(D).to(torch.bfloat16)
+    wq[4] = 3e38
+    wk = torch.ones(D).to(torch.bfloat16)
+    tab = _table(S, rot)
+    gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, False, 1e-6)
+    assert np.array_equal(gq, rq)
+    assert np.array_equal(gk, rk)
+
+
+@pytest.mark.parametrize("D,rot,inter", [(128, 128, False), (256, 256, True), (64, 0, False)])
+def test_prologue_many_tokens_bit_exact(sk, D, rot, inter):
+    """Several blocks of tokens and a ragged last block (tokens not a multiple
+    of the tokens per block), ordinary values: bit-identical to the oracle."""
+    gen = torch.Generator().manual_seed(D + rot)
+    B, S, Hq, Hkv = 3, 171, 7, 1
+    q = (torch.randn(B, S, Hq, D, generator=gen) * 3).to(torch.bfloat16)
+    k = (torch.randn(B, S, Hkv, D, generator=gen) * 0.2).to(torch.bfloat16)
+    wq = (1 + 0.2 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (0.5 + 0.2 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    tab = _table(S, rot) if rot else torch.zeros(S, 0)
+    gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, inter, 1e-5)
+    assert np.array_equal(gq, rq)
+    assert np.array_equal(gk, rk)
+
+
+@pytest.mark.parametrize("inter,scale", [(False, 1.0), (True, 1e-3), (False, 300.0)])
+def test_prologue_large_bit_exact(sk, inter, scale):
+    """About 5M elements per call: enough that a few thousand elements land
+    near a bf16 midpoint and take the kernel's fp64 fix-up; every output bit
+    equals the oracle's."""
+    gen = torch.Generator().manual_seed(int(scale * 7) + int(inter))
+    B, S, Hq, Hkv, D, rot = 1, 4096, 8, 2, 128, 128
+    q = (torch.randn(B, S, Hq, D, generator=gen) * scale).to(torch.bfloat16)
+    k = (torch.randn(B, S, Hkv, D, generator=gen) * scale).to(torch.bfloat16)
+    wq = (1 + 0.3 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (0.7 + 0.3 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    tab = _table(S, rot, theta=1e6)
+    gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, inter, 1e-6)
+    assert np.array_equal(gq, rq), np.argwhere(gq != rq)[:5]
+    assert np.array_equal(gk, rk), np.argwhere(gk != rk)[:5]
