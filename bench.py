@@ -41,6 +41,7 @@ KERNEL_SOURCES = ["varlen_flash_attention_b200/csrc/attn_fwd_sm100.cuh",
                   "varlen_flash_attention_b200/csrc/ptx.cuh",
                   "varlen_flash_attention_b200/csrc/splitkv_attn.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+PROLOGUE_SOURCES = ["varlen_flash_attention_b200/csrc/qk_norm_rope.cuh"]
 
 
 def q_valid_of(w):
@@ -57,12 +58,24 @@ def flops_of(w, rows=None):
     return 4.0 * w.D * w.Hq * sum(q * n for q, n in zip(qv, rl))
 
 
-def kernel_source_sha():
+def kernel_source_sha(sources=None):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in (KERNEL_SOURCES if sources is None else sources):
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def captured_traffic(key, sources=None):
+    """DRAM bytes of one launch from profiles/traffic.json, or None when the
+    entry is missing or the kernel sources changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        e = json.load(f).get(key)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha(sources):
+        return None
+    return int(e["dram_bytes_per_launch"])
 
 
 SUSTAINED_AFTER_S = 1.0  # a timed region longer than this runs under the power cap
@@ -83,14 +96,7 @@ def measured_peaks(timed_s: float = 0.0):
 
 
 def traffic_per_launch(workload):
-    if not os.path.exists(TRAFFIC_FILE):
-        return None
-    with open(TRAFFIC_FILE) as f:
-        d = json.load(f)
-    e = d.get(workload)
-    if not e or e.get("kernel_source_sha") != kernel_source_sha():
-        return None
-    return e.get("dram_bytes_per_launch")
+    return captured_traffic(workload)
 
 
 class ClockSampler:
@@ -421,7 +427,8 @@ def run_prologue(args, w):
     torch.cuda.set_device(dev)
     g = torch.Generator().manual_seed(w.seed)
     S = w.Sq
-    n_copies = 2
+    per_copy = 2 * w.B * S * (w.Hq + w.Hkv) * w.D  # q + k bytes
+    n_copies = max(2, -(-2 * 126 * 2 ** 20 // per_copy))  # rotating copies > 2x L2
     qs = [torch.randn(w.B, S, w.Hq, w.D, generator=g).to(torch.bfloat16).to(dev) for _ in range(n_copies)]
     ks = [torch.randn(w.B, S, w.Hkv, w.D, generator=g).to(torch.bfloat16).to(dev) for _ in range(n_copies)]
     wq = torch.ones(w.D, dtype=torch.bfloat16, device=dev)
@@ -451,9 +458,9 @@ def run_prologue(args, w):
         "dtype": "bf16 in/out, fp64 arithmetic", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.B, "seq": S, "heads_q": w.Hq, "heads_kv": w.Hkv,
                    "head_dim": w.D, "rot_dim": rot, "bytes_per_step": nbytes,
-                   "l2": f"{n_copies} rotating q/k copies"},
+                   "l2": f"{n_copies} rotating q/k copies, {n_copies * per_copy / 1e6:.0f} MB > 2x L2"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                     "peak_kind": kind, "traffic": None},
+                     "peak_kind": kind, "traffic": captured_traffic("prologue:" + w.name, PROLOGUE_SOURCES)},
         "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
     return 0
 

@@ -188,3 +188,20 @@ def test_prologue_large_bit_exact(sk, inter, scale):
     gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, inter, 1e-6)
     assert np.array_equal(gq, rq), np.argwhere(gq != rq)[:5]
     assert np.array_equal(gk, rk), np.argwhere(gk != rk)[:5]
+
+
+@pytest.mark.parametrize("D,inter", [(128, False), (64, True)])
+def test_prologue_many_heads_bit_exact(sk, D, inter):
+    """32 heads per token (20 q + 12 k) walked by one lane group, two rows
+    at a time across the q/k boundary, ragged last block; every output bit
+    equals the oracle's."""
+    gen = torch.Generator().manual_seed(40 + D)
+    B, S, Hq, Hkv, rot = 2, 100, 20, 12, D
+    q = torch.randn(B, S, Hq, D, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, S, Hkv, D, generator=gen).to(torch.bfloat16)
+    wq = (1 + 0.2 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (1 + 0.2 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    tab = _table(S, rot)
+    gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, inter, 1e-6)
+    assert np.array_equal(gq, rq), np.argwhere(gq != rq)[:5]
+    assert np.array_equal(gk, rk), np.argwhere(gk != rk)[:5]
