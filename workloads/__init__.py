@@ -88,6 +88,12 @@ WORKLOADS: Dict[str, Workload] = {
             real_len=(25048,), seed=4,
             description="long GQA self attention: 512 + 24576 keys, last 40 suffix tokens are pad",
         ),
+        Workload(
+            "pad_heavy", B=1, Hq=16, Hkv=16, D=128, Sq=8192, Sp=512, Ss=8192,
+            real_len=(4608,), seed=6,
+            description="pad-exclusion evidence: the last 4096 of 8192 suffix keys are tail pad "
+                        "(DRAM reads must be Q + the valid K/V only)",
+        ),
     ]
 }
 
