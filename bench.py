@@ -455,7 +455,7 @@ def run_prologue(args, w):
     print(json.dumps({
         "metric": "qk_rmsnorm_rope (A0 prologue) HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "dtype": "bf16 in/out, fp64 arithmetic", "data": "synthetic",
+        "dtype": "f32 (sum of squares, r and undecided bf16 roundings in f64)", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.B, "seq": S, "heads_q": w.Hq, "heads_kv": w.Hkv,
                    "head_dim": w.D, "rot_dim": rot, "bytes_per_step": nbytes,
                    "l2": f"{n_copies} rotating q/k copies, {n_copies * per_copy / 1e6:.0f} MB > 2x L2"},
