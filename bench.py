@@ -207,8 +207,11 @@ def combine_ranks(flop_per_step, steps, dt_ms, dist, device="cuda"):
     return dt_max, total / (dt_max / 1e3) / 1e12
 
 
-def cpu_oracle_sample(w, target_s=10.0, seed=0):
-    """Time the fp64 oracle on a bounded row sample of the workload (host cores)."""
+def cpu_oracle_sample(w, gpu_out=None, target_s=10.0, seed=0):
+    """Time the fp64 oracle on a bounded row sample of the workload (host cores).
+
+    With ``gpu_out`` (the kernel's output on the same inputs), also compare the
+    sampled rows with it: (cpu_baseline dict, oracle_check dict)."""
     import numpy as np
 
     import oracle
@@ -224,12 +227,24 @@ def cpu_oracle_sample(w, target_s=10.0, seed=0):
     n2 = int(min(w.Sq, max(n, n * target_s / max(dt, 1e-3))))
     rows = sorted(int(r) for r in rng.choice(w.Sq, size=n2, replace=False))
     t0 = time.perf_counter()
-    oracle.attn_split_kv(**t, real_len=rl, rows=rows)
+    ref = oracle.attn_split_kv(**t, real_len=rl, rows=rows)
     dt = time.perf_counter() - t0
     fl = flops_of(w, rows)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(rows)} of {w.Sq} query rows x {w.Hq} heads x {w.B} batch rows of {w.name} "
-                      f"({fl / 1e9:.1f} GFLOP, {dt:.1f} s)"}
+    cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": f"{len(rows)} of {w.Sq} query rows x {w.Hq} heads x {w.B} batch rows of {w.name} "
+                     f"({fl / 1e9:.1f} GFLOP, {dt:.1f} s)"}
+    if gpu_out is None:
+        return cpu, None
+    got = gpu_out[:, rows].float().cpu().numpy().astype(np.float64)
+    diff = got - ref
+    max_abs = float(np.abs(diff).max())
+    rel_l2 = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+    qv = q_valid_of(w)
+    pad_zero = all(bool((gpu_out[b, qv[b]:] == 0).all()) for b in range(w.B))
+    check = {"max_abs": max_abs, "rel_l2": rel_l2, "rows": f"{len(rows)} of {w.Sq} x {w.Hq} heads x {w.B}",
+             "bound": {"max_abs": 2e-2, "rel_l2": 1e-2}, "pad_rows_exactly_zero": pad_zero,
+             "pass": max_abs <= 2e-2 and rel_l2 <= 1e-2 and pad_zero}
+    return cpu, check
 
 
 def run_reference(args, w):
@@ -380,7 +395,8 @@ def run_ours(args, w):
     clocks = clk.summary()
     line = None
     if rank == 0:
-        cpu = cpu_oracle_sample(w) if world == 1 and not args.no_cpu_baseline else None
+        cpu, check = (cpu_oracle_sample(w, outs[0]) if world == 1 and not args.no_cpu_baseline
+                      else (None, None))
         line = {
             "metric": METRIC,
             "value": value,
@@ -402,6 +418,7 @@ def run_ours(args, w):
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "traffic": traffic_per_launch(w.name)},
             "cpu_baseline": cpu,
+            "oracle_check": check,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps,
