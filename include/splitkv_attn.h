@@ -55,7 +55,7 @@ extern "C" {
 typedef enum {
   SK_OK = 0,
   SK_ERR_INVALID_ARG = 1,    /* bad sizes, strides, alignment, ranges, aliasing */
-  SK_ERR_UNSUPPORTED = 2,    /* valid request this build does not serve (head_dim, device) */
+  SK_ERR_UNSUPPORTED = 2,    /* valid request the library does not serve (head_dim, device) */
   SK_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed */
   SK_ERR_DEVICE_TIMEOUT = 4  /* a kernel gave up a bounded wait (see sk_device_status) */
 } sk_status_t;
