@@ -205,3 +205,18 @@ def test_prologue_many_heads_bit_exact(sk, D, inter):
     gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, inter, 1e-6)
     assert np.array_equal(gq, rq), np.argwhere(gq != rq)[:5]
     assert np.array_equal(gk, rk), np.argwhere(gk != rk)[:5]
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(3, 2, 128), (2, 1, 64), (5, 4, 256)])
+def test_prologue_odd_head_count_bit_exact(sk, Hq, Hkv, D):
+    """An odd number of rows per token: the last batch of two holds one row."""
+    gen = torch.Generator().manual_seed(Hq * 10 + Hkv + D)
+    B, S, rot = 2, 37, D // 2 if D != 64 else 64
+    q = torch.randn(B, S, Hq, D, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, S, Hkv, D, generator=gen).to(torch.bfloat16)
+    wq = (1 + 0.2 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (1 + 0.2 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    tab = _table(S, rot)
+    gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, False, 1e-6)
+    assert np.array_equal(gq, rq), np.argwhere(gq != rq)[:5]
+    assert np.array_equal(gk, rk), np.argwhere(gk != rk)[:5]
