@@ -115,6 +115,43 @@ SK_API sk_status_t attn_fwd_split_kv_ex(const sk_tensor_t* q, const sk_tensor_t*
                                  const int32_t* q_valid, void* stream);
 
 /*
+ * attn_fwd_split_kv_scatter — as attn_fwd_split_kv_ex, with the output
+ * all-to-all of the Ulysses form fused into the store ("sglang PR 26973",
+ * _forward_with_replicated_kv_prefix_split: head-sharded attention, then an
+ * all-to-all of the output from head shards back to sequence shards).  The
+ * query stream is the gathered sequence of num_dst equal chunks; output row s
+ * of batch row b and (local) query head h is written to
+ *
+ *   dst[s / L] + b*dst_layout.stride_b + (s % L)*dst_layout.stride_s
+ *              + (head_offset + h)*dst_layout.stride_h,   L = dst_layout.len_s
+ *
+ * i.e. straight into the receive buffer of the rank that owns that chunk, at
+ * this rank's head slot.  Each tile's rows are stored as soon as the tile is
+ * done, so the exchange overlaps the attention of later tiles.
+ *
+ *   dst        HOST array of num_dst (1..8) device addresses, 16-byte aligned.
+ *              They may be other GPUs' memory mapped into this process (CUDA
+ *              IPC, symmetric memory); the kernel issues only plain stores to
+ *              them and ends with a system-scope fence.  The caller owns the
+ *              buffers and must order the readers after this call (e.g. a
+ *              barrier across ranks once the stream reaches it).
+ *   dst_layout strides of every destination (ptr ignored); len_s = L, and
+ *              num_dst * L must equal q.len_s.  Heads head_offset ..
+ *              head_offset + num_q_heads - 1 of each destination are written
+ *              (pad rows as zeros); nothing else is touched.
+ * Destinations are not checked for overlap with the inputs (they may live on
+ * other devices); the caller keeps them apart.  Other arguments and errors as
+ * attn_fwd_split_kv_ex.
+ */
+SK_API sk_status_t attn_fwd_split_kv_scatter(const sk_tensor_t* q, const sk_tensor_t* k_prefix,
+                                      const sk_tensor_t* v_prefix, const sk_tensor_t* k_suffix,
+                                      const sk_tensor_t* v_suffix, const int32_t* real_len,
+                                      const int32_t* q_valid, int32_t num_q_heads, int32_t num_kv_heads,
+                                      float softmax_scale, void* const* dst, int32_t num_dst,
+                                      const sk_tensor_t* dst_layout, int32_t head_offset, int32_t batch,
+                                      int32_t head_dim, void* stream);
+
+/*
  * attn_fwd_varlen — packed variable-length attention: several independent
  * sequences (segments) concatenated along one token axis, each attending only
  * to its own keys (a block-diagonal mask, never materialised).  Sources:

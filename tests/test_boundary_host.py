@@ -234,3 +234,39 @@ def test_shard_pad_copy_rejects_bad_arguments(L, kw):
                              a["dst_ss"], a["dst_rows"], a["first_row"], a["row_bytes"], a["batch"],
                              a["pad_mode"], None)
     assert st == INVALID, (st, L.sk_last_error())
+
+
+def _scatter(L, n=2, chunk=32, ptrs=None, head_offset=0, layout=None, Hq=2, D=64, Sq=64):
+    g = _good(D=D, H=Hq, Sq=Sq)
+    if ptrs is None:
+        ptrs = [FAKE + ((6 + r) << 24) for r in range(n)]
+    arr = (ctypes.c_void_p * max(1, len(ptrs)))(*ptrs) if ptrs else None
+    if layout is None:
+        layout = _t(chunk, chunk * 4 * Hq * D, 4 * Hq * D, D, None)
+    return L.attn_fwd_split_kv_scatter(
+        *[ctypes.byref(x) for x in g[:5]], None, None, Hq, Hq, 0.125,
+        ctypes.cast(arr, ctypes.c_void_p) if arr is not None else None, n, ctypes.byref(layout),
+        head_offset, 1, D, None)
+
+
+@pytest.mark.parametrize("kw", [
+    {"n": 0}, {"n": 9, "chunk": 8},                       # 1..8 destinations
+    {"n": 2, "chunk": 31},                                # 2 x 31 != 64 query rows
+    {"ptrs": [FAKE + (6 << 24), None]},                   # NULL destination
+    {"ptrs": [FAKE + (6 << 24), FAKE + (7 << 24) + 8]},   # misaligned destination
+    {"head_offset": -1},
+    {"layout": _t(32, 32 * 512, 508, 64, None)},          # stride_s not a multiple of 8
+    {"layout": _t(32, 32 * 512, 64, 64, None)},           # rows of 2 heads overlap
+])
+def test_scatter_rejects_bad_arguments(L, kw):
+    st = _scatter(L, **kw)
+    assert st == INVALID, (st, L.sk_last_error())
+    assert L.sk_last_error()
+
+
+def test_scatter_rejects_null_destination_array(L):
+    g = _good()
+    layout = _t(32, 32 * 512, 512, 64, None)
+    st = L.attn_fwd_split_kv_scatter(*[ctypes.byref(x) for x in g[:5]], None, None, 2, 2, 0.125, None, 2,
+                                     ctypes.byref(layout), 0, 1, 64, None)
+    assert st == INVALID

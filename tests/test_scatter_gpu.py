@@ -1,0 +1,82 @@
+"""Fused output all-to-all (attn_fwd_split_kv_scatter) on one GPU.
+
+The Ulysses form ("sglang PR 26973", _forward_with_replicated_kv_prefix_split)
+runs attention on a rank's head shard over the whole gathered sequence, then
+an all-to-all returns each sequence chunk to the rank that owns it.  Here
+every rank's receive buffer is a tensor on this GPU: each emulated rank calls
+the scatter entry on its heads, writing straight into all ranks' buffers, and
+the buffers must equal the chunks of the plain kernel's output bit for bit
+(each (query tile, head) is computed the same way in both launches).  The
+cross-GPU form (peer-mapped buffers, a barrier before the readers) needs
+several GPUs and is not run here.
+"""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = 7.0
+
+
+@pytest.fixture(scope="module")
+def sk():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from varlen_flash_attention_b200 import build
+
+    build.build()
+    import varlen_flash_attention_b200 as m
+
+    return m
+
+
+@pytest.mark.parametrize("sp,L,Hq,Hkv,D,B,pad", [
+    (2, 256, 4, 4, 128, 1, 0),      # chunks aligned to 128-row tiles
+    (2, 200, 4, 2, 128, 1, 0),      # tiles straddle the chunk boundary, GQA
+    (4, 77, 8, 2, 64, 2, 5),        # 4 chunks, tail pad on the last rank's chunk, B = 2
+    (8, 33, 8, 8, 128, 1, 9),       # one head per rank, short chunks, tail pad
+])
+def test_scatter_equals_plain_output_chunks(sk, sp, L, Hq, Hkv, D, B, pad):
+    g = torch.Generator().manual_seed(sp * 100 + L)
+    Sq = sp * L
+    Sp = 48
+    dev = "cuda"
+
+    def r(*shape):
+        return torch.randn(*shape, generator=g).to(torch.bfloat16).to(dev)
+
+    q, kp, vp = r(B, Sq, Hq, D), r(B, Sp, Hkv, D), r(B, Sp, Hkv, D)
+    ks, vs = r(B, Sq, Hkv, D), r(B, Sq, Hkv, D)
+    real_len = [Sp + Sq - pad] * B
+    q_valid = [Sq - pad] * B
+    ref = sk.attn_fwd_split_kv(q, kp, vp, ks, vs, real_len=real_len, q_valid=q_valid)
+    # receive buffers: [B, L, Hq + 2 canary heads, D], canaries hold SENTINEL
+    recv = [torch.full((B, L, Hq + 2, D), SENTINEL, dtype=torch.bfloat16, device=dev) for _ in range(sp)]
+    hl = Hq // sp  # query heads per rank; its KV heads are the ones they read (q head h reads h // group)
+    for rank in range(sp):
+        h0 = rank * hl
+        kv0 = h0 // (Hq // Hkv)
+        sl = slice(kv0, kv0 + max(1, hl // (Hq // Hkv)))
+        sk.attn_fwd_split_kv_scatter(q[:, :, h0:h0 + hl], kp[:, :, sl], vp[:, :, sl], ks[:, :, sl], vs[:, :, sl],
+                                     recv, head_offset=h0, real_len=real_len, q_valid=q_valid)
+    torch.cuda.synchronize()
+    for rank in range(sp):
+        got = recv[rank]
+        want = ref[:, rank * L:(rank + 1) * L]
+        assert torch.equal(got[:, :, :Hq].view(torch.int16), want.view(torch.int16)), rank
+        assert bool((got[:, :, Hq:] == SENTINEL).all()), "canary heads written"
+    if pad:
+        assert bool((recv[-1][:, L - pad:, :Hq] == 0).all())
+    assert sk.sk_device_status(0) == 0
+
+
+def test_scatter_single_destination_is_the_plain_call(sk):
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(1, 300, 2, 128, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(1, 260, 2, 128, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(1, 260, 2, 128, generator=g).to(torch.bfloat16).cuda()
+    ref = sk.attn_fwd_split_kv(q, k[:, :60], v[:, :60], k[:, 60:], v[:, 60:], real_len=[250])
+    out = torch.empty_like(ref)
+    sk.attn_fwd_split_kv_scatter(q, k[:, :60], v[:, :60], k[:, 60:], v[:, 60:], [out], real_len=[250])
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))

@@ -26,6 +26,7 @@ __all__ = [
     "SkTensor",
     "lib",
     "attn_fwd_split_kv",
+    "attn_fwd_split_kv_scatter",
     "attn_fwd_varlen",
     "sk_shard_pad_copy",
     "qk_rmsnorm_rope",
@@ -82,6 +83,9 @@ def lib() -> ctypes.CDLL:
             L.attn_fwd_split_kv_ex.argtypes = [P, P, P, P, P, vp, i32, i32, ctypes.c_float, P, i32, i32,
                                                vp, vp]
             L.attn_fwd_split_kv_ex.restype = i32
+            L.attn_fwd_split_kv_scatter.argtypes = [P, P, P, P, P, vp, vp, i32, i32, ctypes.c_float, vp, i32,
+                                                    P, i32, i32, i32, vp]
+            L.attn_fwd_split_kv_scatter.restype = i32
             i64 = ctypes.c_int64
             L.sk_shard_pad_copy.argtypes = [vp, i64, i64, i32, vp, i64, i64, i32, i32, i32, i32, i32, vp]
             L.sk_shard_pad_copy.restype = i32
@@ -175,6 +179,49 @@ def attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix,
         st = L.attn_fwd_split_kv_ex(*args, ctypes.cast(qv, ctypes.c_void_p), _stream_ptr(stream))
     _check(st)
     return out
+
+
+def attn_fwd_split_kv_scatter(q, k_prefix, v_prefix, k_suffix, v_suffix, dst: Sequence,
+                              head_offset: int = 0, real_len: Optional[Sequence[int]] = None,
+                              softmax_scale: Optional[float] = None,
+                              q_valid: Optional[Sequence[int]] = None, stream=None) -> None:
+    """``attn_fwd_split_kv`` with the output all-to-all fused into the store.
+
+    The query stream is the gathered sequence of ``len(dst)`` equal chunks;
+    output row s goes to ``dst[s // L][:, s % L, head_offset:head_offset + Hq]``
+    with L = ``dst[r].shape[1]``.  ``dst``: 1..8 bf16 tensors of one shape and
+    one stride set ([B, L, H_total, D]), e.g. the ranks' receive buffers mapped
+    into this process (peer memory).  The caller orders their readers after
+    this call (a barrier across ranks).
+    """
+    B, Sq, Hq, D = q.shape
+    Hkv = k_prefix.shape[2] if k_prefix.shape[1] > 0 else k_suffix.shape[2]
+    dst = list(dst)
+    if not 1 <= len(dst) <= 8:
+        raise ValueError("1 to 8 destinations")
+    shape, strides = tuple(dst[0].shape), dst[0].stride()
+    for t in dst[1:]:
+        if tuple(t.shape) != shape or t.stride() != strides:
+            raise ValueError("destinations differ in shape or strides")
+    if len(shape) != 4 or shape[0] != B or shape[3] != D or shape[1] * len(dst) != Sq:
+        raise ValueError(f"destinations {shape} x {len(dst)} do not hold [B={B}, Sq={Sq}, *, D={D}]")
+    if head_offset < 0 or head_offset + Hq > shape[2]:
+        raise ValueError(f"heads {head_offset}..{head_offset + Hq - 1} outside the destination's {shape[2]}")
+    if softmax_scale is None:
+        softmax_scale = D ** -0.5
+    descs = [tensor_desc(t) for t in (q, k_prefix, v_prefix, k_suffix, v_suffix)]
+    layout = tensor_desc(dst[0])
+    ptrs = (ctypes.c_void_p * len(dst))(*[t.data_ptr() for t in dst])
+    rl = _int32_array(real_len, B)
+    qv = _int32_array(q_valid, B)
+    L = lib()
+    st = L.attn_fwd_split_kv_scatter(
+        *[ctypes.byref(d) for d in descs],
+        ctypes.cast(rl, ctypes.c_void_p) if rl is not None else None,
+        ctypes.cast(qv, ctypes.c_void_p) if qv is not None else None,
+        Hq, Hkv, float(softmax_scale), ctypes.cast(ptrs, ctypes.c_void_p), len(dst), ctypes.byref(layout),
+        int(head_offset), B, D, _stream_ptr(stream))
+    _check(st)
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int],

@@ -86,6 +86,7 @@ constexpr int kTilesPerCta = 2;  // query tiles per CTA
 constexpr int kRowsPerCta = kBlockM * kTilesPerCta;
 constexpr int kBlockN = 128;     // keys per KV tile
 constexpr int kMaxBatch = 8;     // batch rows per launch (tensor maps live in parameter space)
+constexpr int kMaxOutDst = 8;    // destinations of a scattered output (ranks of one node)
 constexpr int kTmaWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
@@ -105,9 +106,15 @@ struct alignas(64) AttnParams {
   int32_t n_prefix[kMaxBatch];  // valid prefix keys = min(Sp, real_len)
   int32_t n_suffix[kMaxBatch];  // valid suffix keys = max(0, real_len - Sp)
   int32_t sq[kMaxBatch];        // output rows of the entry (rows in [q_valid, sq) are written as zeros)
-  int64_t out_off[kMaxBatch];   // element offset of the entry's row 0, head 0 from `out`
+  int64_t out_off[kMaxBatch];   // element offset of the entry's row 0, head 0 from `out` (or a destination)
   uint16_t* out;
   int64_t out_ss, out_sh;
+  // Scattered output (out_chunk > 0): row s goes to out_dst[s / out_chunk] at
+  // row s % out_chunk, e.g. the receive buffers of the ranks that own each
+  // sequence chunk (the output all-to-all of the Ulysses form).  The pointers
+  // may address peer GPUs' memory; only plain stores are issued to them.
+  int32_t out_chunk;
+  uint16_t* out_dst[kMaxOutDst];
   int32_t group;                // num_q_heads / num_kv_heads
   float scale_log2;             // softmax_scale * log2(e)
   int32_t* status;              // device status word
@@ -194,14 +201,28 @@ struct Waiter {
   }
 };
 
-__device__ __forceinline__ void store_zero_rows(uint16_t* base, int64_t ss, int r_begin,
+// Address of output row `row` of entry `bl`, query head `hq` (kScatter: the
+// row's destination buffer, see AttnParams::out_chunk).
+template <bool kScatter>
+__device__ __forceinline__ uint16_t* out_row_ptr(const AttnParams& p, int bl, int hq, int row) {
+  const int64_t head = static_cast<int64_t>(hq) * p.out_sh;
+  if constexpr (!kScatter) {
+    return p.out + p.out_off[bl] + head + static_cast<int64_t>(row) * p.out_ss;
+  } else {
+    const int rk = row / p.out_chunk;
+    return p.out_dst[rk] + p.out_off[bl] + head + static_cast<int64_t>(row - rk * p.out_chunk) * p.out_ss;
+  }
+}
+
+template <bool kScatter>
+__device__ __forceinline__ void store_zero_rows(const AttnParams& p, int bl, int hq, int r_begin,
                                                 int r_end, int D, int tid, int nthreads) {
   const int chunks = D / 8;  // 16-byte chunks per row
   const int total = (r_end - r_begin) * chunks;
   for (int idx = tid; idx < total; idx += nthreads) {
     const int r = r_begin + idx / chunks;
     const int c = idx % chunks;
-    *reinterpret_cast<uint4*>(base + static_cast<int64_t>(r) * ss + c * 8) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(out_row_ptr<kScatter>(p, bl, hq, r) + c * 8) = make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -302,7 +323,7 @@ __device__ __forceinline__ void store_p_row(uint32_t p_base, int r, const uint32
   }
 }
 
-template <int D>
+template <int D, bool kScatter = false>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams p) {
   using L = SmemLayout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -322,12 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   const int tS = (nks + kBlockN - 1) / kBlockN;
   const int n_tiles = tP + tS;
   const int sq = p.sq[bl];
-  uint16_t* out_bh = p.out + p.out_off[bl] + static_cast<int64_t>(hq) * p.out_sh;
+  uint16_t* out_bh = p.out + p.out_off[bl] + static_cast<int64_t>(hq) * p.out_sh;  // plain output only
 
   if (row0 >= qv || n_tiles == 0) {
     // Every row of this CTA is pad, or this batch row has no valid key: exact zeros.
     const int r_end = min(row0 + kRowsPerCta, sq);
-    store_zero_rows(out_bh, p.out_ss, row0, r_end, D, threadIdx.x, kThreads);
+    store_zero_rows<kScatter>(p, bl, hq, row0, r_end, D, threadIdx.x, kThreads);
+    if constexpr (kScatter) __threadfence_system();
     return;
   }
 
@@ -645,7 +667,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const int row = row0 + x * kBlockM + r;
-      uint16_t* orow = out_bh + static_cast<int64_t>(row) * p.out_ss;
+      uint16_t* orow = kScatter ? out_row_ptr<true>(p, bl, hq, row < sq ? row : 0)
+                                : out_bh + static_cast<int64_t>(row) * p.out_ss;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -673,6 +696,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
   }
 
+  // scattered rows may sit in peer memory: order them before whatever signal
+  // the caller raises after the kernel (a barrier across ranks)
+  if constexpr (kScatter) __threadfence_system();
   skptx::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

@@ -54,7 +54,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sm_count = 0;
   int32_t* status = nullptr;
-  bool attn_attr_set[2] = {false, false};
+  bool attn_attr_set[4] = {false, false, false, false};  // (D 64, D 128) x (plain, scattered)
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -185,24 +185,36 @@ template <int D>
 sk_status_t launch_attn(const skattn::AttnParams& prm, int n_qtiles, int H, int nb, cudaStream_t stream,
                         DeviceInfo* dev) {
   using L = skattn::SmemLayout<D>;
-  const int slot = (D == 64) ? 0 : 1;
+  const bool scatter = prm.out_chunk > 0;  // separate instance: the plain kernel's code is untouched
+  const int slot = (D == 64 ? 0 : 1) + (scatter ? 2 : 0);
+  auto kernel = scatter ? skattn::attn_fwd_kernel<D, true> : skattn::attn_fwd_kernel<D, false>;
   if (!dev->attn_attr_set[slot]) {
-    cudaError_t e = cudaFuncSetAttribute(skattn::attn_fwd_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     dev->attn_attr_set[slot] = true;
   }
   dim3 grid(n_qtiles, H, nb);
-  skattn::attn_fwd_kernel<D><<<grid, skattn::kThreads, L::kAlloc, stream>>>(prm);
+  kernel<<<grid, skattn::kThreads, L::kAlloc, stream>>>(prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return SK_OK;
 }
 
+// Output rows scattered over destination buffers (the output all-to-all of
+// the Ulysses form): row s -> dst[s / layout.len_s], row s % layout.len_s,
+// head head_offset + h; every destination has layout's strides.
+struct ScatterOut {
+  void* const* dst;
+  int32_t n;
+  const sk_tensor_t* layout;
+  int32_t head_offset;
+};
+
 sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tensor_t* vp,
                       const sk_tensor_t* ks, const sk_tensor_t* vs, const int32_t* real_len,
                       int32_t Hq, int32_t Hkv, float scale, const sk_tensor_t* out, int32_t B,
-                      int32_t D, const int32_t* q_valid_in, void* stream_v) {
+                      int32_t D, const int32_t* q_valid_in, void* stream_v,
+                      const ScatterOut* scatter = nullptr) {
   if (B < 0) return fail(SK_ERR_INVALID_ARG, "batch < 0");
   if (Hq <= 0 || Hkv <= 0) return fail(SK_ERR_INVALID_ARG, "head counts must be positive");
   if (Hq % Hkv != 0) return fail(SK_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
@@ -215,22 +227,46 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
   if ((st = check_tensor("v_prefix", vp, B, Hkv, D)) != SK_OK) return st;
   if ((st = check_tensor("k_suffix", ks, B, Hkv, D)) != SK_OK) return st;
   if ((st = check_tensor("v_suffix", vs, B, Hkv, D)) != SK_OK) return st;
-  if ((st = check_tensor("out", out, B, Hq, D)) != SK_OK) return st;
   const int32_t Sq = q->len_s;
-  if (out->len_s != Sq) return fail(SK_ERR_INVALID_ARG, "out.len_s (%d) != q.len_s (%d)", out->len_s, Sq);
+  sk_tensor_t scatter_view;  // one destination as a tensor, for the stride checks
+  if (scatter) {
+    if (scatter->n < 1 || scatter->n > skattn::kMaxOutDst)
+      return fail(SK_ERR_INVALID_ARG, "num_dst=%d outside [1, %d]", scatter->n, skattn::kMaxOutDst);
+    if (!scatter->dst || !scatter->layout) return fail(SK_ERR_INVALID_ARG, "NULL destination array or layout");
+    if (scatter->head_offset < 0) return fail(SK_ERR_INVALID_ARG, "head_offset < 0");
+    const int32_t chunk = scatter->layout->len_s;
+    if (chunk <= 0 || static_cast<int64_t>(chunk) * scatter->n != Sq)
+      return fail(SK_ERR_INVALID_ARG, "num_dst (%d) x dst rows (%d) != q.len_s (%d)", scatter->n, chunk, Sq);
+    for (int r = 0; r < scatter->n; ++r) {
+      if (!scatter->dst[r]) return fail(SK_ERR_INVALID_ARG, "destination %d is NULL", r);
+      if (reinterpret_cast<uintptr_t>(scatter->dst[r]) % 16)
+        return fail(SK_ERR_INVALID_ARG, "destination %d not 16-byte aligned", r);
+    }
+    scatter_view = *scatter->layout;
+    scatter_view.ptr = scatter->dst[0];
+    if ((st = check_tensor("dst", &scatter_view, B, scatter->head_offset + Hq, D)) != SK_OK) return st;
+    if (!no_self_overlap(scatter_view, B, scatter->head_offset + Hq, D))
+      return fail(SK_ERR_INVALID_ARG, "destination layout overlaps itself");
+    out = &scatter_view;
+  } else {
+    if ((st = check_tensor("out", out, B, Hq, D)) != SK_OK) return st;
+    if (out->len_s != Sq) return fail(SK_ERR_INVALID_ARG, "out.len_s (%d) != q.len_s (%d)", out->len_s, Sq);
+  }
   if (kp->len_s != vp->len_s) return fail(SK_ERR_INVALID_ARG, "k_prefix.len_s != v_prefix.len_s");
   if (ks->len_s != vs->len_s) return fail(SK_ERR_INVALID_ARG, "k_suffix.len_s != v_suffix.len_s");
   const int64_t Sp = kp->len_s, Ss = ks->len_s, Skv = Sp + Ss;
   if (Skv > INT32_MAX) return fail(SK_ERR_INVALID_ARG, "Sp + Ss too large");
-  if (!no_self_overlap(*out, B, Hq, D)) return fail(SK_ERR_INVALID_ARG, "out overlaps itself");
+  if (!scatter && !no_self_overlap(*out, B, Hq, D)) return fail(SK_ERR_INVALID_ARG, "out overlaps itself");
   if (B == 0 || Sq == 0) return SK_OK;
-  Span so, si;
-  span_of(*out, B, Hq, D, &so);
-  const struct { const char* n; const sk_tensor_t* t; int H; } ins[5] = {
-      {"q", q, Hq}, {"k_prefix", kp, Hkv}, {"v_prefix", vp, Hkv}, {"k_suffix", ks, Hkv}, {"v_suffix", vs, Hkv}};
-  for (auto& in : ins) {
-    span_of(*in.t, B, in.H, D, &si);
-    if (overlaps(so, si)) return fail(SK_ERR_INVALID_ARG, "out overlaps %s", in.n);
+  if (!scatter) {  // destinations of a scattered output may live on other GPUs: the caller keeps them apart
+    Span so, si;
+    span_of(*out, B, Hq, D, &so);
+    const struct { const char* n; const sk_tensor_t* t; int H; } ins[5] = {
+        {"q", q, Hq}, {"k_prefix", kp, Hkv}, {"v_prefix", vp, Hkv}, {"k_suffix", ks, Hkv}, {"v_suffix", vs, Hkv}};
+    for (auto& in : ins) {
+      span_of(*in.t, B, in.H, D, &si);
+      if (overlaps(so, si)) return fail(SK_ERR_INVALID_ARG, "out overlaps %s", in.n);
+    }
   }
   for (int b = 0; b < B; ++b) {
     const int64_t n = real_len ? real_len[b] : Skv;
@@ -275,9 +311,16 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
         if ((st = encode_map(&prm.tm_vs[i], bptr(vs), vs->stride_s, vs->stride_h, Hkv, nsuf, D)) != SK_OK) return st;
       }
     }
-    prm.out = static_cast<uint16_t*>(out->ptr) + static_cast<int64_t>(b0) * out->stride_b;
     prm.out_ss = out->stride_s;
     prm.out_sh = out->stride_h;
+    if (scatter) {
+      prm.out_chunk = out->len_s;
+      for (int r = 0; r < scatter->n; ++r)
+        prm.out_dst[r] = static_cast<uint16_t*>(scatter->dst[r]) + static_cast<int64_t>(b0) * out->stride_b +
+                         static_cast<int64_t>(scatter->head_offset) * out->stride_h;
+    } else {
+      prm.out = static_cast<uint16_t*>(out->ptr) + static_cast<int64_t>(b0) * out->stride_b;
+    }
     prm.group = Hq / Hkv;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.status = info->status;
@@ -396,6 +439,22 @@ sk_status_t attn_fwd_split_kv(const sk_tensor_t* q, const sk_tensor_t* k_prefix,
   try {
     return attn_impl(q, k_prefix, v_prefix, k_suffix, v_suffix, real_len, num_q_heads, num_kv_heads,
                      softmax_scale, out, batch, head_dim, nullptr, stream);
+  } catch (...) {
+    return fail(SK_ERR_INVALID_ARG, "internal exception");
+  }
+}
+
+sk_status_t attn_fwd_split_kv_scatter(const sk_tensor_t* q, const sk_tensor_t* k_prefix,
+                                      const sk_tensor_t* v_prefix, const sk_tensor_t* k_suffix,
+                                      const sk_tensor_t* v_suffix, const int32_t* real_len,
+                                      const int32_t* q_valid, int32_t num_q_heads, int32_t num_kv_heads,
+                                      float softmax_scale, void* const* dst, int32_t num_dst,
+                                      const sk_tensor_t* dst_layout, int32_t head_offset, int32_t batch,
+                                      int32_t head_dim, void* stream) {
+  try {
+    const ScatterOut sc{dst, num_dst, dst_layout, head_offset};
+    return attn_impl(q, k_prefix, v_prefix, k_suffix, v_suffix, real_len, num_q_heads, num_kv_heads,
+                     softmax_scale, nullptr, batch, head_dim, q_valid, stream, &sc);
   } catch (...) {
     return fail(SK_ERR_INVALID_ARG, "internal exception");
   }
