@@ -80,3 +80,23 @@ def test_scatter_single_destination_is_the_plain_call(sk):
     sk.attn_fwd_split_kv_scatter(q, k[:, :60], v[:, :60], k[:, 60:], v[:, 60:], [out], real_len=[250])
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
+def test_fused_ulysses_single_rank_uses_the_scatter_kernel(sk):
+    """ulysses_attn_fwd_split_kv_fused at sp = 1 (no process group): the
+    scatter kernel writes the output into the rank's own receive buffer."""
+    from varlen_flash_attention_b200 import sp_shard as sps
+    from varlen_flash_attention_b200 import ulysses
+
+    g = torch.Generator().manual_seed(9)
+    B, S, Hq, Hkv, D, Sp = 1, 333, 8, 2, 128, 64
+    mk = lambda *sh: torch.randn(*sh, generator=g).to(torch.bfloat16).cuda()
+    q, ks, vs = mk(B, S, Hq, D), mk(B, S, Hkv, D), mk(B, S, Hkv, D)
+    kp, vp = mk(B, Sp, Hkv, D), mk(B, Sp, Hkv, D)
+    plan = sps.build_shard_plan(S, 1, 0)
+    recv = [torch.full((B, S, Hq, D), SENTINEL, dtype=torch.bfloat16, device="cuda")]
+    out = ulysses.ulysses_attn_fwd_split_kv_fused(q, kp, vp, ks, vs, plan, recv)
+    ref = ulysses.ulysses_attn_fwd_split_kv(q, kp, vp, ks, vs, plan)
+    torch.cuda.synchronize()
+    assert out.data_ptr() == recv[0].data_ptr()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))

@@ -24,6 +24,13 @@ Q heads by more than 1.5x.
 The collectives are ``torch.distributed.all_to_all_single`` (NCCL over
 NVLink/NVSwitch on GPUs); the attention itself is the CUDA kernel unless a
 ``local_attn`` callable with the same signature is supplied.
+
+``ulysses_attn_fwd_split_kv_fused`` fuses step 4 into the kernel: its
+epilogue stores every output row straight into the receive buffer of the rank
+that owns the row's sequence chunk (``attn_fwd_split_kv_scatter``: plain
+stores to buffers mapped from the other GPUs, e.g. torch symmetric memory),
+so the exchange overlaps the attention of later tiles; a barrier across the
+group then orders the readers after every rank's stores.
 """
 from __future__ import annotations
 
@@ -35,7 +42,8 @@ import torch.nn.functional as F
 
 from .sp_shard import SpShard
 
-__all__ = ["seq_to_head", "head_to_seq", "gqa_head_padding", "ulysses_attn_fwd_split_kv"]
+__all__ = ["seq_to_head", "head_to_seq", "gqa_head_padding", "ulysses_attn_fwd_split_kv",
+           "ulysses_attn_fwd_split_kv_fused"]
 
 _warned_inflation = False
 
@@ -100,12 +108,27 @@ def ulysses_attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix, shard: 
     [B, S_local, Hq, D]; its pad rows are zeros.
     """
     sp = shard.sp_size
+    Hq, D = q.shape[2], q.shape[3]
+    if local_attn is None:
+        from . import attn_fwd_split_kv as local_attn
+    # q_valid: the query stream is the suffix stream, so its tail pad rows are pad too
+    qh, kp, vp, ksh, vsh, real_len, q_valid, _ = _head_shard_inputs(
+        q, k_prefix, v_prefix, k_suffix, v_suffix, shard, group, suffix_real_len)
+    if softmax_scale is None:
+        softmax_scale = D ** -0.5
+    oh = local_attn(qh, kp, vp, ksh, vsh, real_len=real_len, q_valid=q_valid, softmax_scale=softmax_scale)
+    out = head_to_seq(oh, sp, group)
+    return out[:, :, :Hq]
+
+
+def _head_shard_inputs(q, k_prefix, v_prefix, k_suffix, v_suffix, shard, group, suffix_real_len):
+    """Steps 1-3 of the split path: exchanged Q / K/V suffix on this rank's
+    heads, the prefix head slice, and the per-row lengths."""
+    sp = shard.sp_size
     B, S_loc, Hq, D = q.shape
     Hkv = k_suffix.shape[2]
     if S_loc != shard.local_len or k_suffix.shape[1] != S_loc or v_suffix.shape[1] != S_loc:
         raise ValueError("q / k_suffix / v_suffix are not this rank's chunk of the plan")
-    if local_attn is None:
-        from . import attn_fwd_split_kv as local_attn
     Hq_p, Hkv_p = gqa_head_padding(Hq, Hkv, sp)
     global _warned_inflation
     if Hq_p > 1.5 * Hq and not _warned_inflation:
@@ -121,10 +144,40 @@ def ulysses_attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix, shard: 
     vp = _pad_heads(v_prefix, Hkv_p)[:, :, h0:h0 + hkv_loc]
     Sp = k_prefix.shape[1]
     srl = [shard.orig_len] * B if suffix_real_len is None else [int(x) for x in suffix_real_len]
-    real_len = [Sp + n for n in srl]
-    q_valid = srl  # the query stream is the suffix stream: its tail pad rows are pad
+    return qh, kp, vp, ksh, vsh, [Sp + n for n in srl], srl, Hq_p
+
+
+def ulysses_attn_fwd_split_kv_fused(q, k_prefix, v_prefix, k_suffix, v_suffix, shard: SpShard,
+                                    recv_buffers: Sequence, group=None,
+                                    softmax_scale: Optional[float] = None,
+                                    suffix_real_len: Optional[Sequence[int]] = None,
+                                    local_attn_scatter: Optional[Callable] = None):
+    """``ulysses_attn_fwd_split_kv`` with the output all-to-all fused into the
+    attention kernel's stores.
+
+    recv_buffers: ``sp`` tensors [B, S_local, Hq_p, D] (Hq_p = the padded query
+    head count of ``gqa_head_padding``); entry r is rank r's receive buffer as
+    mapped into this process (another GPU's memory, e.g. a torch symmetric
+    memory buffer; entry ``sp_rank`` is this rank's own).  This rank's heads
+    land at head slot ``sp_rank * Hq_p / sp`` of every buffer.  After the
+    kernel a barrier over ``group`` orders this rank's read of its own buffer
+    after every rank's stores.  Returns this rank's output chunk [B, S_local,
+    Hq, D] (a view of its receive buffer; pad rows are zeros).
+    """
+    import torch.distributed as dist
+
+    sp = shard.sp_size
+    if len(recv_buffers) != sp:
+        raise ValueError(f"{len(recv_buffers)} receive buffers for {sp} ranks")
+    if local_attn_scatter is None:
+        from . import attn_fwd_split_kv_scatter as local_attn_scatter
+    Hq, D = q.shape[2], q.shape[3]
+    qh, kp, vp, ksh, vsh, real_len, q_valid, Hq_p = _head_shard_inputs(
+        q, k_prefix, v_prefix, k_suffix, v_suffix, shard, group, suffix_real_len)
     if softmax_scale is None:
         softmax_scale = D ** -0.5
-    oh = local_attn(qh, kp, vp, ksh, vsh, real_len=real_len, q_valid=q_valid, softmax_scale=softmax_scale)
-    out = head_to_seq(oh, sp, group)
-    return out[:, :, :Hq]
+    local_attn_scatter(qh, kp, vp, ksh, vsh, list(recv_buffers), head_offset=shard.sp_rank * (Hq_p // sp),
+                       real_len=real_len, q_valid=q_valid, softmax_scale=softmax_scale)
+    if sp > 1:
+        dist.barrier(group=group)
+    return recv_buffers[shard.sp_rank][:, :, :Hq]
