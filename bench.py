@@ -482,6 +482,62 @@ def run_prologue(args, w):
     return 0
 
 
+def run_scatter(args, w):
+    """The attention with its output scattered over ``args.scatter`` destination
+    buffers on this GPU (the stores of the fused output all-to-all; on several
+    GPUs the buffers would be the ranks' receive buffers): TFLOP/s against
+    the same roofline as the plain line."""
+    import varlen_flash_attention_b200 as sk
+
+    n = args.scatter
+    if w.Sq % n:
+        raise SystemExit(f"{w.name}: Sq={w.Sq} does not split into {n} chunks")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    rl = w.real_lens()
+    n_copies = 4
+    host = workloads.make_inputs(w)
+    keys = ("q", "k_prefix", "v_prefix", "k_suffix", "v_suffix")
+    copies = [{k: host[k].to(dev) for k in keys} for _ in range(n_copies)]
+    dsts = [[torch.empty(w.B, w.Sq // n, w.Hq, w.D, dtype=torch.bfloat16, device=dev) for _ in range(n)]
+            for _ in range(n_copies)]
+
+    def step(i):
+        c = copies[i % n_copies]
+        sk.attn_fwd_split_kv_scatter(c["q"], c["k_prefix"], c["v_prefix"], c["k_suffix"], c["v_suffix"],
+                                     dsts[i % n_copies], real_len=rl)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        e0.record()
+        for i in range(args.steps):
+            step(i)
+        e1.record()
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    fl = flops_of(w)
+    value = fl / (ms / 1e3) / 1e12
+    peak, peak_kind = measured_peaks(ms * args.steps / 1e3)
+    ref = sk.attn_fwd_split_kv(copies[0]["q"], copies[0]["k_prefix"], copies[0]["v_prefix"],
+                               copies[0]["k_suffix"], copies[0]["v_suffix"], real_len=rl)
+    torch.cuda.synchronize(dev)
+    same = all(torch.equal(d.view(torch.int16), ref[:, r * (w.Sq // n):(r + 1) * (w.Sq // n)].view(torch.int16))
+               for r, d in enumerate(dsts[0]))
+    print(json.dumps({
+        "metric": METRIC + " (output scattered over destination buffers)", "value": value, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "out_scatter": n, "rows_per_destination": w.Sq // n,
+                   "l2": "inputs rotate over 4 device copies (> 126 MB L2)"},
+        "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                     "peak_kind": peak_kind, "traffic": None},
+        "scattered_equals_plain_output": same, "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -492,11 +548,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["attention", "prologue"], default="attention",
                     help="prologue: time the optional fused Q/K RMSNorm+RoPE kernel instead")
+    ap.add_argument("--scatter", type=int, default=0,
+                    help="N > 1: scatter the attention output over N destination buffers (fused all-to-all stores)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = workloads.get(args.workload)
     if args.op == "prologue":
         return run_prologue(args, w)
+    if args.scatter > 1:
+        return run_scatter(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -132,9 +132,11 @@ SK_API sk_status_t attn_fwd_split_kv_ex(const sk_tensor_t* q, const sk_tensor_t*
  *   dst        HOST array of num_dst (1..8) device addresses, 16-byte aligned.
  *              They may be other GPUs' memory mapped into this process (CUDA
  *              IPC, symmetric memory); the kernel issues only plain stores to
- *              them and ends with a system-scope fence.  The caller owns the
- *              buffers and must order the readers after this call (e.g. a
- *              barrier across ranks once the stream reaches it).
+ *              them, all performed by the time it completes in stream order.
+ *              The caller owns the buffers and orders the readers after that
+ *              point: a barrier across ranks enqueued on `stream` after this
+ *              call (an NCCL collective signals its peers only after the work
+ *              before it on the stream has completed).
  *   dst_layout strides of every destination (ptr ignored); len_s = L, and
  *              num_dst * L must equal q.len_s.  Heads head_offset ..
  *              head_offset + num_q_heads - 1 of each destination are written

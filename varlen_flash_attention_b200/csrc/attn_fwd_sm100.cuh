@@ -112,7 +112,10 @@ struct alignas(64) AttnParams {
   // Scattered output (out_chunk > 0): row s goes to out_dst[s / out_chunk] at
   // row s % out_chunk, e.g. the receive buffers of the ranks that own each
   // sequence chunk (the output all-to-all of the Ulysses form).  The pointers
-  // may address peer GPUs' memory; only plain stores are issued to them.
+  // may address peer GPUs' memory; only plain stores are issued to them, and
+  // they are performed by the time the kernel completes (no per-CTA fence: a
+  // CTA exits while its stores drain, and the caller's barrier after the
+  // kernel publishes them).
   int32_t out_chunk;
   uint16_t* out_dst[kMaxOutDst];
   int32_t group;                // num_q_heads / num_kv_heads
@@ -349,7 +352,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // Every row of this CTA is pad, or this batch row has no valid key: exact zeros.
     const int r_end = min(row0 + kRowsPerCta, sq);
     store_zero_rows<kScatter>(p, bl, hq, row0, r_end, D, threadIdx.x, kThreads);
-    if constexpr (kScatter) __threadfence_system();
     return;
   }
 
@@ -696,9 +698,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
   }
 
-  // scattered rows may sit in peer memory: order them before whatever signal
-  // the caller raises after the kernel (a barrier across ranks)
-  if constexpr (kScatter) __threadfence_system();
   skptx::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
