@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import varlen_flash_attention_b200 as sk
 from varlen_flash_attention_b200 import SkTensor, build
@@ -270,3 +271,19 @@ def test_scatter_rejects_null_destination_array(L):
     st = L.attn_fwd_split_kv_scatter(*[ctypes.byref(x) for x in g[:5]], None, None, 2, 2, 0.125, None, 2,
                                      ctypes.byref(layout), 0, 1, 64, None)
     assert st == INVALID
+
+
+def test_scatter_binding_checks_shapes_before_the_library():
+    q = torch.zeros(1, 64, 2, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 16, 2, 64, dtype=torch.bfloat16)
+    good = [torch.zeros(1, 32, 4, 64, dtype=torch.bfloat16) for _ in range(2)]
+    with pytest.raises(ValueError):
+        sk.attn_fwd_split_kv_scatter(q, kv, kv, kv, kv, [])                      # no destination
+    with pytest.raises(ValueError):
+        sk.attn_fwd_split_kv_scatter(q, kv, kv, kv, kv, good * 5)                # 10 destinations
+    with pytest.raises(ValueError):
+        sk.attn_fwd_split_kv_scatter(q, kv, kv, kv, kv, [good[0], good[1][:, :16]])  # shapes differ
+    with pytest.raises(ValueError):
+        sk.attn_fwd_split_kv_scatter(q, kv, kv, kv, kv, good[:1])                # 1 x 32 rows != 64
+    with pytest.raises(ValueError):
+        sk.attn_fwd_split_kv_scatter(q, kv, kv, kv, kv, good, head_offset=3)     # heads 3..4 of 4
