@@ -538,6 +538,36 @@ def run_scatter(args, w):
     return 0
 
 
+def run_host(args, w):
+    """Host cost of one call (validation, per-row metadata, five tensor-map
+    encodings, launch) on a workload whose kernel is far shorter than that:
+    wall time of back-to-back calls, which the host then bounds."""
+    import varlen_flash_attention_b200 as sk
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    t = {k: v.to(dev) for k, v in workloads.make_inputs(w).items()}
+    out = torch.empty(w.B, w.Sq, w.Hq, w.D, dtype=torch.bfloat16, device=dev)
+    rl = w.real_lens()
+    call = lambda: sk.attn_fwd_split_kv(t["q"], t["k_prefix"], t["v_prefix"], t["k_suffix"], t["v_suffix"],
+                                        real_len=rl, out=out)
+    for _ in range(max(args.warmup, 50)):
+        call()
+    torch.cuda.synchronize(dev)
+    n = max(args.steps, 2000)
+    t0 = time.perf_counter()
+    for _ in range(n):
+        call()
+    t1 = time.perf_counter()
+    torch.cuda.synchronize(dev)
+    t2 = time.perf_counter()
+    print(json.dumps({"metric": "host cost per attn_fwd_split_kv call (Python binding + C ABI + launch)",
+                      "value": (t1 - t0) / n * 1e6, "unit": "us", "calls": n, "higher_is_better": False,
+                      "drain_after_last_call_us": (t2 - t1) * 1e6,
+                      "config": {"workload": w.name}}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -546,8 +576,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["attention", "prologue"], default="attention",
-                    help="prologue: time the optional fused Q/K RMSNorm+RoPE kernel instead")
+    ap.add_argument("--op", choices=["attention", "prologue", "host"], default="attention",
+                    help="prologue: time the optional fused Q/K RMSNorm+RoPE kernel instead; "
+                         "host: host cost of one attention call (tiny workload)")
     ap.add_argument("--scatter", type=int, default=0,
                     help="N > 1: scatter the attention output over N destination buffers (fused all-to-all stores)")
     args = ap.parse_args()
@@ -555,6 +586,8 @@ def main():
     w = workloads.get(args.workload)
     if args.op == "prologue":
         return run_prologue(args, w)
+    if args.op == "host":
+        return run_host(args, w)
     if args.scatter > 1:
         return run_scatter(args, w)
     if args.impl == "reference":
