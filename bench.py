@@ -540,9 +540,12 @@ def run_scatter(args, w):
 
 def run_host(args, w):
     """Host cost of one call (validation, per-row metadata, five tensor-map
-    encodings, launch) on a workload whose kernel is far shorter than that:
-    wall time of back-to-back calls, which the host then bounds."""
+    encodings, launch) on the tiny workload, whose kernel is far shorter than
+    that: wall time of back-to-back calls, which the host then bounds
+    (``--workload`` is ignored: a longer kernel would bound the loop instead)."""
     import varlen_flash_attention_b200 as sk
+
+    w = workloads.get("tiny")
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -578,7 +581,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["attention", "prologue", "host"], default="attention",
                     help="prologue: time the optional fused Q/K RMSNorm+RoPE kernel instead; "
-                         "host: host cost of one attention call (tiny workload)")
+                         "host: host cost of one attention call (always the tiny workload)")
     ap.add_argument("--scatter", type=int, default=0,
                     help="N > 1: scatter the attention output over N destination buffers (fused all-to-all stores)")
     args = ap.parse_args()
