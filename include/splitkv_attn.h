@@ -137,8 +137,8 @@ SK_API sk_status_t attn_fwd_split_kv_ex(const sk_tensor_t* q, const sk_tensor_t*
  *              point: a barrier across ranks enqueued on `stream` after this
  *              call (an NCCL collective signals its peers only after the work
  *              before it on the stream has completed).
- *   dst_layout strides of every destination (ptr ignored); len_s = L, and
- *              num_dst * L must equal q.len_s.  Heads head_offset ..
+ *   dst_layout strides of every destination (ptr ignored); len_s = L >= 1,
+ *              and num_dst * L must equal q.len_s.  Heads head_offset ..
  *              head_offset + num_q_heads - 1 of each destination are written
  *              (pad rows as zeros); nothing else is touched.
  * Destinations are not checked for overlap with the inputs (they may live on

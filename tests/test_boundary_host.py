@@ -287,3 +287,19 @@ def test_scatter_binding_checks_shapes_before_the_library():
         sk.attn_fwd_split_kv_scatter(q, kv, kv, kv, kv, good[:1])                # 1 x 32 rows != 64
     with pytest.raises(ValueError):
         sk.attn_fwd_split_kv_scatter(q, kv, kv, kv, kv, good, head_offset=3)     # heads 3..4 of 4
+
+
+def test_scatter_empty_batch_is_a_no_op(L):
+    """batch 0 succeeds without touching the device, like the plain entry
+    (an empty query stream is rejected instead: destinations have >= 1 row)."""
+    g = _good()
+    layout = _t(32, 32 * 256, 256, 64, None)
+    arr = (ctypes.c_void_p * 2)(FAKE + (6 << 24), FAKE + (7 << 24))
+    st = L.attn_fwd_split_kv_scatter(*[ctypes.byref(x) for x in g[:5]], None, None, 2, 2, 0.125,
+                                     ctypes.cast(arr, ctypes.c_void_p), 2, ctypes.byref(layout), 0, 0, 64, None)
+    assert st == 0, L.sk_last_error()
+    g = _good(Sq=0)
+    layout = _t(0, 0, 256, 64, None)
+    st = L.attn_fwd_split_kv_scatter(*[ctypes.byref(x) for x in g[:5]], None, None, 2, 2, 0.125,
+                                     ctypes.cast(arr, ctypes.c_void_p), 2, ctypes.byref(layout), 0, 1, 64, None)
+    assert st == 1
