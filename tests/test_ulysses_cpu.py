@@ -172,3 +172,14 @@ def test_head_padding_rule():
     assert ulysses.gqa_head_padding(6, 3, 4) == (8, 4)
     with pytest.raises(ValueError):
         ulysses.gqa_head_padding(6, 4, 2)
+
+
+def test_fused_form_needs_one_receive_buffer_per_rank():
+    from varlen_flash_attention_b200 import sp_shard as sps
+    from varlen_flash_attention_b200 import ulysses
+
+    plan = sps.build_shard_plan(10, 2, 0)
+    x = torch.zeros(1, plan.local_len, 2, 64)
+    kv = torch.zeros(1, 3, 2, 64)
+    with pytest.raises(ValueError):
+        ulysses.ulysses_attn_fwd_split_kv_fused(x, kv, kv, x, x, plan, [torch.zeros(1, 5, 2, 64)])
