@@ -1,10 +1,12 @@
 """Benchmark of split-KV tail-padded attention on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload cosmos_self]
+                    [--workload long_gqa]
 
 A step is one call of attn_fwd_split_kv over one batch of the workload (the
-whole hot path: one kernel).  Inputs are synthetic (seeded, see workloads/)
+whole hot path: one kernel).  The default workload is the largest one
+(long GQA self-attention: B 1, Hq 32 / Hkv 8, D 128, 512 prefix + 24576
+suffix keys of which the last 40 are tail pad).  Inputs are synthetic (seeded, see workloads/)
 and rotate over 4 device copies (> 126 MB L2) so no step reads another step's
 data from L2.  Device time is measured with CUDA events on the launching
 stream, W warm-up steps first, barrier + synchronize on both sides, max over
@@ -35,7 +37,7 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "split-KV attention TFLOP/s and % of B200 dense-bf16 peak; max-abs err vs CPU oracle"
-DEFAULT_WORKLOAD = "cosmos_self"
+DEFAULT_WORKLOAD = "long_gqa"
 FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["varlen_flash_attention_b200/csrc/attn_fwd_sm100.cuh",
                   "varlen_flash_attention_b200/csrc/ptx.cuh",
@@ -56,6 +58,36 @@ def flops_of(w, rows=None):
     if rows is not None:
         qv = [sum(1 for r in rows if r < qv[b]) for b in range(w.B)]
     return 4.0 * w.D * w.Hq * sum(q * n for q, n in zip(qv, rl))
+
+
+def hbm_bytes_of(w):
+    """Algorithmic DRAM bytes of one call: the valid query rows read once,
+    the valid K/V rows read once per (batch row, KV head), every output row
+    written once (pad rows as zeros)."""
+    rl = w.real_lens()
+    qv = q_valid_of(w)
+    row = w.D * 2
+    q = sum(qv) * w.Hq * row
+    kv = 2 * sum(rl) * w.Hkv * row
+    o = w.B * w.Sq * w.Hq * row
+    return q + kv + o
+
+
+def forced_rows(w):
+    """Rows every oracle check includes: the first row, the rows on either
+    side of the prefix/suffix boundary, the last valid query row and every
+    pad query row."""
+    qv = min(q_valid_of(w))
+    rows = {0, w.Sp - 1, w.Sp, qv - 1} | set(range(qv, w.Sq))
+    return sorted(r for r in rows if 0 <= r < w.Sq)
+
+
+def measured_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured copy"
+    return 6650.0, "fallback copy"
 
 
 def kernel_source_sha(sources=None):
@@ -225,7 +257,7 @@ def cpu_oracle_sample(w, gpu_out=None, target_s=10.0, seed=0):
     oracle.attn_split_kv(**t, real_len=rl, rows=rows)
     dt = time.perf_counter() - t0
     n2 = int(min(w.Sq, max(n, n * target_s / max(dt, 1e-3))))
-    rows = sorted(int(r) for r in rng.choice(w.Sq, size=n2, replace=False))
+    rows = sorted(set(int(r) for r in rng.choice(w.Sq, size=n2, replace=False)) | set(forced_rows(w)))
     t0 = time.perf_counter()
     ref = oracle.attn_split_kv(**t, real_len=rl, rows=rows)
     dt = time.perf_counter() - t0
@@ -241,7 +273,9 @@ def cpu_oracle_sample(w, gpu_out=None, target_s=10.0, seed=0):
     rel_l2 = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
     qv = q_valid_of(w)
     pad_zero = all(bool((gpu_out[b, qv[b]:] == 0).all()) for b in range(w.B))
-    check = {"max_abs": max_abs, "rel_l2": rel_l2, "rows": f"{len(rows)} of {w.Sq} x {w.Hq} heads x {w.B}",
+    check = {"max_abs": max_abs, "rel_l2": rel_l2,
+             "rows": f"{len(rows)} of {w.Sq} x {w.Hq} heads x {w.B} (seeded sample + forced rows "
+                     f"0, prefix/suffix boundary, last valid, all pad)",
              "bound": {"max_abs": 2e-2, "rel_l2": 1e-2}, "pad_rows_exactly_zero": pad_zero,
              "pass": max_abs <= 2e-2 and rel_l2 <= 1e-2 and pad_zero}
     return cpu, check
@@ -392,6 +426,9 @@ def run_ours(args, w):
         raise RuntimeError("end-to-end output differs from the device-timed output")
 
     peak, peak_kind = measured_peaks(dt_ms_max / 1e3)
+    hbm_peak, hbm_kind = measured_hbm()
+    hbm_b = hbm_bytes_of(w)
+    hbm_gbs = hbm_b / (per_launch_ms / 1e3) / 1e9
     clocks = clk.summary()
     line = None
     if rank == 0:
@@ -417,6 +454,9 @@ def run_ours(args, w):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "traffic": traffic_per_launch(w.name)},
+            "hbm": {"bytes_per_step": hbm_b, "achieved": hbm_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": hbm_gbs / hbm_peak, "peak_kind": hbm_kind,
+                    "bytes": "valid Q rows + valid K/V once per KV head + every output row"},
             "cpu_baseline": cpu,
             "oracle_check": check,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -574,8 +614,8 @@ def run_host(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -195,6 +195,53 @@ def attn_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int
     return out
 
 
+def shard_chunk(x, orig_len: int, sp_size: int, sp_rank: int, pad_mode: str = "zeros",
+                mutate: str = "") -> np.ndarray:
+    """One rank's chunk of an even, tail-padded sequence shard, along axis 1.
+
+    Definition ("sglang PR 30107", sp_shard_utils.py: build_shard_plan's
+    shard math and shard_like's pad-then-narrow): a stream of ``orig_len``
+    rows is cut into ``sp_size`` chunks of ``local_len = ceil(orig_len /
+    sp_size)`` rows; the ``local_len * sp_size - orig_len`` missing rows are
+    appended after the last real row, as zeros or (``pad_mode="repeat_last"``)
+    as copies of the last real row; rank ``r`` holds padded rows
+    ``[r * local_len, (r + 1) * local_len)``.  Written row by row: padded row
+    t is source row t when t < orig_len, else the pad row.
+
+    x: [B, orig_len, ...] bf16 tensor (compared as bit patterns) or any numpy
+    array.  Returns a numpy array [B, local_len, ...] (uint16 bits for bf16).
+    ``mutate`` plants a mistake for the pin tests: "floor_len" (local_len
+    rounded down), "pad_first" (pad rows at the chunk head), "repeat_first"
+    (pad repeats row 0).
+    """
+    if hasattr(x, "dtype") and not isinstance(x, np.ndarray):
+        import torch
+
+        a = _bf16_bits(x) if x.dtype == torch.bfloat16 else x.detach().cpu().numpy()
+    else:
+        a = np.asarray(x)
+    if a.shape[1] != orig_len:
+        raise ValueError("axis 1 must hold orig_len rows")
+    if sp_size < 1 or not 0 <= sp_rank < sp_size:
+        raise ValueError("bad sp_size / sp_rank")
+    if pad_mode not in ("zeros", "repeat_last"):
+        raise ValueError("pad_mode")
+    local_len = -(-orig_len // sp_size) if mutate != "floor_len" else orig_len // sp_size
+    num_pad = local_len * sp_size - orig_len
+    out = np.zeros((a.shape[0], local_len) + a.shape[2:], dtype=a.dtype)
+    for r in range(local_len):
+        t = sp_rank * local_len + r
+        if mutate == "pad_first" and sp_rank == sp_size - 1 and num_pad > 0:
+            t = t - num_pad if r >= num_pad else orig_len  # pad rows moved to the chunk head
+        if t < orig_len:
+            out[:, r] = a[:, t]
+        elif pad_mode == "repeat_last":
+            if orig_len == 0:
+                raise ValueError("repeat_last needs a real row")
+            out[:, r] = a[:, 0] if mutate == "repeat_first" else a[:, orig_len - 1]
+    return out
+
+
 def qk_rmsnorm_rope(x, w, table, pos=None, rot_dim: Optional[int] = None,
                     interleaved: bool = False, eps: float = 1e-6) -> np.ndarray:
     """RMSNorm over head_dim then RoPE for x [..., H, D] (bf16); returns bf16 bits (uint16).

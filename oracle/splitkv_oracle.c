@@ -28,7 +28,7 @@
  *    materialisation rule (round to bf16 wherever the unfused path stores
  *    bf16): oracle_qk_rmsnorm_rope.
  *
- * Readings where the pages are silent (each also listed in the design notes):
+ * Readings where the pages are silent:
  *  - GQA: query head hq reads KV head hq / (Hq / Hkv) (contiguous groups).
  *  - Query rows i >= q_valid[b] are pad; their output is exactly 0.
  *  - A row with no valid key (real_len[b] == 0) outputs exactly 0.

@@ -74,45 +74,52 @@ def _check_case(sk, t, real_len=None, q_valid=None, scale=None, rows=None, what=
 # ---------------------------------------------------------------- the five workloads
 
 
-def test_tiny_workload(sk):
+def test_tiny_workload(sk, parity_log):
     w = workloads.get("tiny")
-    _check_case(sk, workloads.make_inputs(w), what="tiny")
+    parity_log("tiny (all rows)", *_check_case(sk, workloads.make_inputs(w), what="tiny"))
 
 
 def _sample_rows(Sq, n, seed, forced=()):
+    """n distinct rows drawn uniformly without replacement (numpy generator
+    seeded with ``seed``), plus the forced rows."""
     g = np.random.default_rng(seed)
     rows = set(int(r) for r in g.choice(Sq, size=min(n, Sq), replace=False))
     rows.update(r for r in forced if 0 <= r < Sq)
     return sorted(rows)
 
 
-def test_cosmos_self_attention(sk):
+# Configs 2-4 are checked on every query row; config 5 on 4096 rows per head
+# (seed 5, uniform without replacement over [0, Sq)) plus rows 0, 511, 512,
+# 25047 and all 40 pad rows.  The same rows serve every head.
+
+
+def test_cosmos_self_attention(sk, parity_log):
     w = workloads.get("cosmos_self")
     t = workloads.make_inputs(w)
-    rows = _sample_rows(w.Sq, 192, 1, forced=(0, 127, 128, 4095))
-    _check_case(sk, t, rows=rows, what="cosmos_self")
+    parity_log("cosmos_self (all rows)", *_check_case(sk, t, what="cosmos_self"))
 
 
-def test_tail_padded_joint(sk):
+def test_tail_padded_joint(sk, parity_log):
     w = workloads.get("tail_padded_joint")
     t = workloads.make_inputs(w)
-    rows = _sample_rows(w.Sq, 160, 2, forced=(0, 4351, 4352, 4428, 4429, 4430, 4431))
-    _check_case(sk, t, real_len=w.real_lens(), rows=rows, what="tail_padded_joint")
+    parity_log("tail_padded_joint (all rows)",
+               *_check_case(sk, t, real_len=w.real_lens(), what="tail_padded_joint"))
 
 
-def test_cross_short_kv(sk):
+def test_cross_short_kv(sk, parity_log):
     w = workloads.get("cross_short_kv")
     t = workloads.make_inputs(w)
-    rows = _sample_rows(w.Sq, 384, 3, forced=(0, 32759, 32639, 32640))
-    _check_case(sk, t, rows=rows, what="cross_short_kv")
+    parity_log("cross_short_kv (all rows)", *_check_case(sk, t, what="cross_short_kv"))
 
 
-def test_long_gqa(sk):
+def test_long_gqa(sk, parity_log):
     w = workloads.get("long_gqa")
     t = workloads.make_inputs(w)
     forced = (0, 511, 512, 25047) + tuple(range(25048, 25088))
-    rows = _sample_rows(w.Sq, 96, 5, forced=forced)
-    _check_case(sk, t, real_len=w.real_lens(), rows=rows, what="long_gqa")
+    rows = _sample_rows(w.Sq, 4096, 5, forced=forced)
+    assert len(rows) >= 4096 and all(r in rows for r in forced)
+    parity_log(f"long_gqa ({len(rows)} rows x 32 heads)",
+               *_check_case(sk, t, real_len=w.real_lens(), rows=rows, what="long_gqa"))
 
 
 # ---------------------------------------------------------------- random shapes, edges

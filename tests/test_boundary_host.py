@@ -303,3 +303,68 @@ def test_scatter_empty_batch_is_a_no_op(L):
     st = L.attn_fwd_split_kv_scatter(*[ctypes.byref(x) for x in g[:5]], None, None, 2, 2, 0.125,
                                      ctypes.cast(arr, ctypes.c_void_p), 2, ctypes.byref(layout), 0, 1, 64, None)
     assert st == 1
+
+
+# ---------------------------------------------------------------- binding shape and device checks
+# Each mismatch must raise ValueError from the binding's own checks (the
+# message names the problem), before any tensor reaches the library.
+
+def _bf(*shape):
+    return torch.zeros(*shape, dtype=torch.bfloat16)
+
+
+def _attn_args(B=2, Sq=64, Hq=4, Hkv=2, D=64, Sp=16, Ss=48):
+    return dict(q=_bf(B, Sq, Hq, D), k_prefix=_bf(B, Sp, Hkv, D), v_prefix=_bf(B, Sp, Hkv, D),
+                k_suffix=_bf(B, Ss, Hkv, D), v_suffix=_bf(B, Ss, Hkv, D))
+
+
+@pytest.mark.parametrize("name, shape, msg", [
+    ("k_prefix", (1, 16, 2, 64), "batch and head_dim"),
+    ("v_suffix", (2, 48, 2, 32), "batch and head_dim"),
+    ("k_suffix", (2, 48, 1, 64), "heads"),
+    ("v_prefix", (2, 16, 4, 64), "heads"),
+    ("v_prefix", (2, 15, 2, 64), "same length"),
+    ("out", (2, 64, 2, 64), "q's shape"),
+    ("out", (1, 64, 4, 64), "q's shape"),
+])
+def test_binding_rejects_shape_mismatch(name, shape, msg, monkeypatch):
+    def no_lib():
+        raise AssertionError("the library must not be reached")
+
+    monkeypatch.setattr(sk, "lib", no_lib)
+    a = _attn_args()
+    a[name] = _bf(*shape)
+    with pytest.raises(ValueError, match=msg):
+        sk.attn_fwd_split_kv(**a)
+
+
+def test_binding_rejects_cpu_weights_and_table_for_prologue(monkeypatch):
+    monkeypatch.setattr(sk, "lib", lambda: (_ for _ in ()).throw(AssertionError("no library call")))
+    q, k = _bf(1, 8, 2, 64), _bf(1, 8, 1, 64)
+    w = _bf(64)
+    tab = torch.zeros(8, 64)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sk.qk_rmsnorm_rope(q, k, w, w, tab)
+    with pytest.raises(ValueError, match="columns"):
+        sk.qk_rmsnorm_rope(q, k, w, w, tab, rot_dim=32)
+    with pytest.raises(ValueError, match="batch, seq and head_dim"):
+        sk.qk_rmsnorm_rope(q, _bf(1, 7, 1, 64), w, w, tab)
+    with pytest.raises(ValueError, match="batch, seq and head_dim"):
+        sk.qk_rmsnorm_rope(q, _bf(2, 8, 1, 64), w, w, tab)
+
+
+def test_prologue_rejects_q_k_sharing_tokens(L):
+    """k placed inside q's token rows (fused layout shifted by one token, or
+    head ranges that spill into the next token) is rejected: the in-place
+    kernel would read and write the same elements from different threads."""
+    D, Hq, Hkv, S = 64, 4, 2, 8
+    ss = (Hq + 2 * Hkv) * D   # fused [B, S, Hq + 2 Hkv, D] row
+    w = FAKE
+    def call(k_off_elems, stride_s=ss):
+        q = _t(S, S * stride_s, stride_s, D)
+        k = _t(S, S * stride_s, stride_s, D, ptr=FAKE + 2 * k_off_elems)
+        return L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, FAKE, S, 64, 0,
+                                 ctypes.c_float(1e-6), Hq, Hkv, 1, D, None)
+    assert call(ss) == 1                  # k = q shifted by one token
+    assert call(Hq * D, stride_s=(Hq + 1) * D) == 1  # k's heads spill into q's next token
+    assert b"overlap" in L.sk_last_error()

@@ -45,41 +45,7 @@
 
 #include "ptx.cuh"
 
-// Build-time switches (defaults are the shipped configuration).
-#ifndef SKA_POLY_EVERY
-#define SKA_POLY_EVERY 0   // k > 0: every k-th score column takes exp2 on the FMA pipe
-#endif
-#ifndef SKA_TRACE
-#define SKA_TRACE 0        // record an event timeline of one CTA (profiling builds only)
-#endif
-#ifndef SKA_ISSUE_SLEEP_NS
-#define SKA_ISSUE_SLEEP_NS 0 // > 0: the MMA issuer naps this long when nothing is ready
-#endif
-#ifndef SKA_WAIT_HINT_NS
-#define SKA_WAIT_HINT_NS 0 // > 0: mbarrier waits ask to be suspended up to this long
-#endif
-
 namespace skattn {
-
-#if SKA_TRACE
-// Event timeline of CTA (SKA_TRACE_CTA, 0, 0): per role, entries of
-// code << 56 | tile << 40 | (clock64 & 2^40-1).
-#ifndef SKA_TRACE_CTA
-#define SKA_TRACE_CTA 1
-#endif
-constexpr int kTraceRoles = 8;
-constexpr int kTraceLen = 8192;
-__device__ unsigned long long g_trace[kTraceRoles][kTraceLen];
-__device__ __forceinline__ void trace(int role, int& idx, int code, int j) {
-  if (blockIdx.x == SKA_TRACE_CTA && blockIdx.y == 0 && blockIdx.z == 0 && idx < kTraceLen)
-    g_trace[role][idx++] = (static_cast<unsigned long long>(code) << 56) |
-                           (static_cast<unsigned long long>(j & 0xFFFF) << 40) |
-                           (static_cast<unsigned long long>(clock64()) & 0xFFFFFFFFFFull);
-}
-#define SKA_TR(role, code, j) trace(role, tr_idx, code, j)
-#else
-#define SKA_TR(role, code, j) ((void)0)
-#endif
 
 constexpr int kBlockM = 128;     // query rows per tile
 constexpr int kTilesPerCta = 2;  // query tiles per CTA
@@ -171,11 +137,7 @@ struct Waiter {
     const uint64_t t0 = skptx::globaltimer_ns();
     uint32_t it = 0;
     while (true) {
-#if SKA_WAIT_HINT_NS > 0
-      if (skptx::mbar_try_wait_hint(bar, parity, SKA_WAIT_HINT_NS)) return true;
-#else
       if (skptx::mbar_try_wait(bar, parity)) return true;
-#endif
       if ((++it & 63u) == 0) {
         if (*abort_flag) return false;
         if (skptx::globaltimer_ns() - t0 > limit_ns) {
@@ -229,29 +191,6 @@ __device__ __forceinline__ void store_zero_rows(const AttnParams& p, int bl, int
   }
 }
 
-// 2^x on the FMA pipe (offloads the MUFU unit).  Cody-Waite split
-// x = n + f, n = nearest integer (added and removed through 1.5 * 2^23),
-// f in [-1/2, 1/2]; p(f) ~= 2^f is the degree-3 minimax polynomial on that
-// interval (relative error 7.5e-5, below the bf16 rounding P gets anyway),
-// coefficients from exp2_poly_fit.py; 2^n is added to p's exponent field.
-// x is clamped at -126 (results there are below 2^-125, i.e. zero for P).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(0.0551716685f, f, 0.2426111251f);
-  p = fmaf(p, f, 0.6932609677f);
-  p = fmaf(p, f, 0.9999280572f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-__device__ __forceinline__ float exp2_col(int c, float x) {
-  if (SKA_POLY_EVERY > 0 && (c % (SKA_POLY_EVERY > 0 ? SKA_POLY_EVERY : 1)) == SKA_POLY_EVERY - 1)
-    return exp2_poly(x);
-  return skptx::ex2_approx(x);
-}
-
 // Valid keys in KV tile j (prefix tiles first, then suffix tiles).
 __device__ __forceinline__ int tile_valid(int j, int tP, int nkp, int nks) {
   return (j < tP) ? min(kBlockN, nkp - j * kBlockN) : min(kBlockN, nks - (j - tP) * kBlockN);
@@ -302,8 +241,8 @@ __device__ __forceinline__ float exp_row_pack(const float (&s)[kBlockN], float s
   for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
 #pragma unroll
   for (int c = 0; c < kBlockN; c += 2) {
-    float e0 = exp2_col(c, fmaf(s[c], sl2, neg_m));
-    float e1 = exp2_col(c + 1, fmaf(s[c + 1], sl2, neg_m));
+    float e0 = skptx::ex2_approx(fmaf(s[c], sl2, neg_m));
+    float e1 = skptx::ex2_approx(fmaf(s[c + 1], sl2, neg_m));
     // exact zeros for masked columns (also when scale == 0, where -inf * 0 is NaN)
     if (PARTIAL && c >= nvalid) e0 = 0.f;
     if (PARTIAL && c + 1 >= nvalid) e1 = 0.f;
@@ -389,9 +328,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
   skptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Waiter W{abort_flag, p.status, p.wait_limit_ns};
-#if SKA_TRACE
-  int tr_idx = 0;
-#endif
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -420,9 +356,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       if (do_k) {
         const int s = j % kKStages;
         if (j >= kKStages && !W.wait_warp(bar(L::bKEmpty + s), ((j / kKStages) - 1) & 1)) { ok = false; break; }
-#if SKA_TRACE
-        if (lane == 0) SKA_TR(1, 42, j);
-#endif
         const CUtensorMap* mk = pre ? &p.tm_kp[bl] : &p.tm_ks[bl];
         skptx::mbar_arrive_expect_tx_elect(bar(L::bKFull + s), L::kKVTile);
 #pragma unroll
@@ -433,9 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       } else {
         const int s = j % kVStages;
         if (j >= kVStages && !W.wait_warp(bar(L::bVEmpty + s), ((j / kVStages) - 1) & 1)) { ok = false; break; }
-#if SKA_TRACE
-        if (lane == 0) SKA_TR(1, 43, j);
-#endif
         const CUtensorMap* mv = pre ? &p.tm_vp[bl] : &p.tm_vs[bl];
         skptx::mbar_arrive_expect_tx_elect(bar(L::bVFull + s), L::kKVTile);
 #pragma unroll
@@ -463,9 +393,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // warp after its loop, so this wait runs out (every role then aborts,
     // drains and exits with SK_ERR_DEVICE_TIMEOUT in the status word).
     if (p.test_stall) ok = ok && W.wait_warp(bar(L::bMmaDone), 0);
-#if SKA_TRACE
-    if (lane == 0) SKA_TR(0, 1, 0);
-#endif
     if (ok) {
       skptx::tc_fence_after();
 #pragma unroll
@@ -496,9 +423,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int j = pN[x];
         if (j < n_tiles && ready(bar(L::bPFull + x), j & 1) &&
             ready(bar(L::bVFull + j % kVStages), (j / kVStages) & 1)) {
-#if SKA_TRACE
-          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 10, j);
-#endif
           skptx::tc_fence_after();
           const int b = x % L::kPBufs;
           issue_pv<D>(tmem + 256 + x * 128, dP + ((b * L::kPTile) >> 4),
@@ -508,25 +432,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
           if (pN[o] > j) skptx::mma_commit_elect(bar(L::bVEmpty + j % kVStages));
           pN[x] = j + 1;
           progressed = true;
-#if SKA_TRACE
-          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 14, j);
-#endif
         }
         const int k = sN[x];
         if (k < n_tiles && ready(bar(L::bSFree + x), (k - 1) & 1) &&
             ready(bar(L::bKFull + k % kKStages), (k / kKStages) & 1)) {
-#if SKA_TRACE
-          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 18, k - 1);
-#endif
           skptx::tc_fence_after();
           issue_s<D>(tmem + x * 128, dQ + ((x * L::kQTile) >> 4), dK + (((k % kKStages) * L::kKVTile) >> 4));
           skptx::mma_commit_elect(bar(L::bSFull + x));
           if (sN[o] > k) skptx::mma_commit_elect(bar(L::bKEmpty + k % kKStages));
           sN[x] = k + 1;
           progressed = true;
-#if SKA_TRACE
-          if (lane == 0) SKA_TR(x == 0 ? 0 : 4, 20, k);
-#endif
         }
       }
       // Bounded: give up once nothing has become ready for the wait limit.
@@ -543,9 +458,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         ok = __all_sync(0xffffffffu, ok);
       }
-#if SKA_ISSUE_SLEEP_NS > 0
-      if (!progressed) __nanosleep(SKA_ISSUE_SLEEP_NS);
-#endif
     }
     // Every MMA this warp issued has finished before TMEM is released.
     skptx::mma_commit_elect(bar(L::bMmaDone));
@@ -560,19 +472,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const int pb = x % L::kPBufs;
     const uint32_t p_base = sbase + L::kP + pb * L::kPTile;
     const float sl2 = p.scale_log2;
-#if SKA_TRACE
-    const bool trl = lane == 0 && (warp % 4) == 0;
-    const int trole = 2 + x;
-#endif
     float m_run = 0.f;  // running (possibly stale) max of scale*log2(e)*s
     float l_run = 0.f;  // running sum of exponentials
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       ok = W.wait_warp(bar(L::bSFull + x), j & 1);
       if (!ok) break;
-#if SKA_TRACE
-      if (trl) SKA_TR(trole, 30, j);
-#endif
       skptx::tc_fence_after();
       float s[kBlockN];
       {
@@ -588,9 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       // S_X(j) is in registers: the issuer may overwrite it with S_X(j+1).
       skptx::tc_fence_before();
       skptx::mbar_arrive(bar(L::bSFree + x));
-#if SKA_TRACE
-      if (trl) SKA_TR(trole, 31, j);
-#endif
       const int nvalid = tile_valid(j, tP, nkp, nks);
       const bool partial = nvalid < kBlockN;
       if (partial) {
@@ -620,9 +522,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       const float sum = partial ? exp_row_pack<true>(s, sl2, -m_run, nvalid, pk)
                                 : exp_row_pack<false>(s, sl2, -m_run, nvalid, pk);
       l_run = l_run * alpha + sum;
-#if SKA_TRACE
-      if (trl) SKA_TR(trole, 32, j);
-#endif
       // Before P_X(j) is stored and before O_X is touched, PV_X(j-1) must have
       // finished.  This also keeps every barrier below within one phase of
       // its waiter (a parity wait cannot tell phase k from k+2).
@@ -659,9 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
       skptx::fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
       skptx::tc_fence_before();
       skptx::mbar_arrive(bar(L::bPFull + x));
-#if SKA_TRACE
-      if (trl) SKA_TR(trole, 35, j);
-#endif
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = W.wait_warp(bar(L::bOReady + x), (n_tiles - 1) & 1);

@@ -566,10 +566,19 @@ sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, const vo
     span_of(*q, batch, num_q_heads, head_dim, &sq);
     span_of(*k, batch, num_kv_heads, head_dim, &sk);
     if (overlaps(sq, sk)) {
-      // allowed only when they are disjoint head ranges of one fused buffer; require distinct elements
-      // by checking that q's heads and k's heads never share an address: same strides, k after q's heads.
-      const bool fused = q->stride_b == k->stride_b && q->stride_s == k->stride_s && q->stride_h == k->stride_h &&
-                         static_cast<const uint16_t*>(k->ptr) >= static_cast<const uint16_t*>(q->ptr) + num_q_heads * q->stride_h;
+      // Allowed only for head ranges of one fused buffer: same strides, k's
+      // first head m whole heads after q's (m >= Hq), and the layout with
+      // m + Hkv heads free of self-overlap, so no element is both a q and a k
+      // element (k shifted by a token, or heads spilling into the next
+      // token, are rejected).
+      const int64_t off = (static_cast<const uint16_t*>(k->ptr) - static_cast<const uint16_t*>(q->ptr));
+      bool fused = q->stride_b == k->stride_b && q->stride_s == k->stride_s && q->stride_h == k->stride_h &&
+                   q->stride_h > 0 && off >= 0 && off % q->stride_h == 0 && off / q->stride_h >= num_q_heads;
+      if (fused) {
+        const int64_t m = off / q->stride_h;
+        fused = m + num_kv_heads <= INT32_MAX &&
+                no_self_overlap(*q, batch, static_cast<int>(m + num_kv_heads), head_dim);
+      }
       if (!fused) return fail(SK_ERR_INVALID_ARG, "q and k overlap");
     }
     if (!w_q || !w_k || (rot_dim > 0 && !rope_table)) return fail(SK_ERR_INVALID_ARG, "NULL weight or table");
@@ -644,14 +653,5 @@ sk_status_t sk_test_stall_mma(int32_t on) {
 
 int32_t sk_abi_version(void) { return kAbiVersion; }
 
-#if SKA_TRACE
-// Profiling builds only: copy the event timeline of the traced CTA to the host.
-SK_API int32_t sk_debug_trace(unsigned long long* host, int32_t n) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  const size_t bytes = sizeof(unsigned long long) * std::min<size_t>(n, skattn::kTraceRoles * skattn::kTraceLen);
-  if (cudaMemcpyFromSymbol(host, skattn::g_trace, bytes) != cudaSuccess) return -1;
-  return 0;
-}
-#endif
 
 }  // extern "C"

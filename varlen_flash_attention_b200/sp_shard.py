@@ -37,33 +37,43 @@ __all__ = [
 
 @dataclass(frozen=True)
 class SpShard:
-    """Facts of one tail-padded even shard, shared by every tensor of a stream."""
+    """An even split of one token stream over ``sp_size`` ranks, as seen by
+    ``sp_rank``.  Hidden states, rotary tables and every other tensor of the
+    stream are cut with the same plan, so their chunks line up.
 
-    orig_len: int   # real tokens (global)
-    local_len: int  # tokens per rank (equal on every rank)
-    num_pad: int    # pad tokens, all at the global tail (the last rank's chunk end)
+    Fields: ``orig_len`` is the count of real tokens in the whole stream;
+    ``local_len`` the chunk length, identical on all ranks; ``num_pad`` the
+    count of filler tokens placed after the last real token (so they end up
+    at the tail of the last chunk); ``sp_size``/``sp_rank`` the group size and
+    this rank's index in it.
+    """
+
+    orig_len: int
+    local_len: int
+    num_pad: int
     sp_size: int
     sp_rank: int
 
     @property
     def local_pad(self) -> int:
-        """Pad rows inside this rank's chunk.  Whenever ``num_pad <= local_len``
-        (every case but tiny sequences over many ranks) this is the page's rule,
-        ``num_pad`` on the last rank and 0 elsewhere.  When the pad outnumbers a
-        chunk (e.g. 1 token over 4 ranks: local_len 1, num_pad 3) it spills into
-        earlier chunks and this counts the pad rows actually inside this one,
-        so ``local_real_len`` never goes negative."""
+        """Filler rows inside this rank's chunk: those of its rows whose global
+        position is at or past ``orig_len``.  While the filler fits in one chunk
+        (``num_pad <= local_len``, i.e. all but tiny streams over many ranks)
+        only the last rank has any, and it has all ``num_pad`` of them.  With
+        more filler than a chunk holds (1 token over 4 ranks: chunks of 1, 3
+        filler rows) the filler reaches into earlier chunks and this still
+        counts the rows that are really there, never a negative real count."""
         end = (self.sp_rank + 1) * self.local_len
         return max(0, min(self.local_len, end - self.orig_len))
 
     @property
     def local_real_len(self) -> int:
-        """Real tokens in this rank's chunk."""
+        """Rows of this rank's chunk that hold real tokens."""
         return self.local_len - self.local_pad
 
     @property
     def padded_len(self) -> int:
-        """Length of the gathered (padded) sequence."""
+        """Rows of the stream once gathered, filler included."""
         return self.local_len * self.sp_size
 
 
@@ -77,12 +87,15 @@ def _group_size_rank(group) -> Tuple[int, int]:
 
 def build_shard_plan(seq_len: int, sp_size: Optional[int] = None, sp_rank: Optional[int] = None,
                      group=None) -> SpShard:
-    """Shard math only, no tensors ("sglang PR 30107", ``build_shard_plan``):
-    ``local_len = ceil(seq_len / sp_size)``, ``num_pad = local_len * sp_size - seq_len``.
+    """Plan the split of a ``seq_len``-token stream; touches no tensor
+    ("sglang PR 30107", ``build_shard_plan``).  Each chunk gets the stream
+    length divided by the group size, rounded up, and the filler is whatever
+    that rounding adds to the total.  One rank (``sp_size == 1``) keeps the
+    stream whole with no filler.
 
     ``sp_size``/``sp_rank`` default to the size and rank of ``group`` (the
     default process group), or to (1, 0) when torch.distributed is not
-    initialised.  With ``sp_size == 1`` the plan is the identity.
+    initialised.
     """
     if sp_size is None or sp_rank is None:
         gs, gr = _group_size_rank(group)
@@ -92,24 +105,27 @@ def build_shard_plan(seq_len: int, sp_size: Optional[int] = None, sp_rank: Optio
         raise ValueError(f"seq_len must be >= 0, got {seq_len}")
     if sp_size < 1 or not (0 <= sp_rank < sp_size):
         raise ValueError(f"bad sp_size/sp_rank: {sp_size}/{sp_rank}")
-    if sp_size == 1:
-        return SpShard(seq_len, seq_len, 0, 1, 0)
-    local_len = (seq_len + sp_size - 1) // sp_size
-    return SpShard(orig_len=seq_len, local_len=local_len, num_pad=local_len * sp_size - seq_len,
-                   sp_size=sp_size, sp_rank=sp_rank)
+    whole, rest = divmod(seq_len, sp_size)
+    chunk = whole + (1 if rest else 0)
+    return SpShard(orig_len=seq_len, local_len=chunk, num_pad=chunk * sp_size - seq_len,
+                   sp_size=sp_size, sp_rank=sp_rank if sp_size > 1 else 0)
 
 
 def tail_attn_meta(shard: SpShard, seqlen_multiplier: int = 1) -> Optional[dict]:
-    """Tail-pad attention metadata of this rank's chunk ("sglang PR 30107",
-    ``tail_attn_meta``): None without pad, else ``valid_len = local_real_len *
-    multiplier`` and ``max_seqlen_tail = max(valid_len, num_pad)`` (the page's
-    fix for the degenerate case where the pad outnumbers the valid tokens).
-    ``seqlen_multiplier`` scales tokens to attention rows (e.g. several rows
-    per token)."""
-    if shard.num_pad == 0:
+    """Attention metadata for this rank's chunk when the stream carries filler
+    ("sglang PR 30107", ``tail_attn_meta``), or None when it carries none.
+    ``valid_len`` counts the attention rows of the chunk's real tokens (each
+    token spans ``seqlen_multiplier`` rows).  ``max_seqlen_tail`` is the longer
+    of that and the filler count: a varlen kernel sized by it then also covers
+    the filler segment, which the page's review found could be the longer of
+    the two."""
+    pad = shard.num_pad
+    if pad <= 0:
         return None
     valid = shard.local_real_len * seqlen_multiplier
-    return {"tail": True, "valid_len": valid, "max_seqlen_tail": max(valid, shard.num_pad)}
+    meta = dict(tail=True, valid_len=valid)
+    meta["max_seqlen_tail"] = valid if valid >= pad else pad
+    return meta
 
 
 def attn_real_len(shard: SpShard, seqlen_multiplier: int = 1, batch: int = 1) -> List[int]:

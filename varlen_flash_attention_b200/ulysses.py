@@ -163,6 +163,15 @@ def ulysses_attn_fwd_split_kv_fused(q, k_prefix, v_prefix, k_suffix, v_suffix, s
     kernel a barrier over ``group`` orders this rank's read of its own buffer
     after every rank's stores.  Returns this rank's output chunk [B, S_local,
     Hq, D] (a view of its receive buffer; pad rows are zeros).
+
+    The returned view is valid only until the next call that uses the same
+    ``recv_buffers``: that call's kernels on the other ranks overwrite the
+    buffer with plain stores as soon as they run.  Every consumer of the
+    result must therefore be enqueued on the calling stream before that next
+    call (the exchange in front of it then orders them), or copy the result
+    out; a consumer on another stream, or a view kept across calls, can see
+    other ranks' newer rows.  Alternating between two buffer sets on
+    consecutive calls gives each result one extra call of lifetime.
     """
     import torch.distributed as dist
 
