@@ -180,6 +180,12 @@ class ClockSampler:
             self.t.start()
         return self
 
+    def mark(self):
+        """Drop what was sampled so far (the summary covers what follows)."""
+        self.samples.clear()
+        self.power_w.clear()
+        self.reasons.clear()
+
     def __exit__(self, *a):
         self._stop.set()
         if self._ok:
@@ -345,16 +351,18 @@ def run_ours(args, w):
         sk.attn_fwd_split_kv(c["q"], c["k_prefix"], c["v_prefix"], c["k_suffix"], c["v_suffix"],
                              real_len=rl, out=outs[i % n_copies], stream=stream)
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
     sk.sk_device_status(local, clear=True)
-
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    # The sampler starts first and the warm-up runs right up to the timed
+    # region: an idle GPU drops its clocks, and the first launch after even a
+    # short idle runs at half speed while they ramp back up.
     with ClockSampler(local) as clk:
+        for i in range(args.warmup):
+            step(i)
         barrier(dist)
         torch.cuda.synchronize(dev)
+        clk.mark()
         ev0.record(stream)
         for i in range(args.steps):
             step(i)
@@ -493,7 +501,8 @@ def run_prologue(args, w):
     rot = w.D
     ang = np.arange(S)[:, None] * 10000.0 ** (-np.arange(0, rot, 2) / rot)
     table = torch.from_numpy(np.concatenate([np.cos(ang), np.sin(ang)], 1).astype(np.float32)).to(dev)
-    step = lambda i: sk.qk_rmsnorm_rope(qs[i % n_copies], ks[i % n_copies], wq, wk, table, rot_dim=rot)
+    step = lambda i: sk.qk_rmsnorm_rope(qs[i % n_copies], ks[i % n_copies], wq, wk, table, rot_dim=rot,
+                                        exact=args.exact)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize(dev)
@@ -512,7 +521,8 @@ def run_prologue(args, w):
     print(json.dumps({
         "metric": "qk_rmsnorm_rope (A0 prologue) HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "dtype": "f32 (sum of squares, r and undecided bf16 roundings in f64)", "data": "synthetic",
+        "dtype": ("f32 (sum of squares, r and undecided bf16 roundings in f64)" if args.exact else "f32"),
+        "data": "synthetic", "instance": "exact" if args.exact else "fp32 (default)",
         "config": {"workload": w.name, "batch": w.B, "seq": S, "heads_q": w.Hq, "heads_kv": w.Hkv,
                    "head_dim": w.D, "rot_dim": rot, "bytes_per_step": nbytes,
                    "l2": f"{n_copies} rotating q/k copies, {n_copies * per_copy / 1e6:.0f} MB > 2x L2"},
@@ -578,6 +588,76 @@ def run_scatter(args, w):
     return 0
 
 
+def run_packed(args, pw):
+    """Packed variable-length attention (attn_fwd_varlen): ``pw.n_seg``
+    samples of unequal length in one call, each attending to itself only.
+    TFLOP/s = 4 * D * Hq * sum(len_i^2) / t, with an oracle check on sampled
+    rows (the first and last row of every segment plus a seeded sample)."""
+    import numpy as np
+
+    import oracle
+    import varlen_flash_attention_b200 as sk
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    t = workloads.make_packed(pw)
+    cu, lens = t["cu_seqlens"], t["lens"]
+    n_copies = 4
+    copies = [{k: t[k].to(dev) for k in ("q", "k", "v")} for _ in range(n_copies)]
+    outs = [torch.empty_like(copies[0]["q"]) for _ in range(n_copies)]
+    fl = 4.0 * pw.D * pw.Hq * sum(float(n) * n for n in lens)
+
+    def step(i):
+        c = copies[i % n_copies]
+        sk.attn_fwd_varlen(c["q"], c["k"], c["v"], cu, cu, out=outs[i % n_copies])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    sk.sk_device_status(0, clear=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(0) as clk:
+        e0.record()
+        for i in range(args.steps):
+            step(i)
+        e1.record()
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    if sk.sk_device_status(0, clear=True) != 0:
+        raise RuntimeError("device status set during the packed run")
+    value = fl / (ms / 1e3) / 1e12
+    peak, peak_kind = measured_peaks(ms * args.steps / 1e3)
+    rng = np.random.default_rng(11)
+    rows = set(rng.choice(cu[-1], size=min(cu[-1], 96), replace=False).tolist())
+    rows |= set(cu[:-1]) | set(c - 1 for c in cu[1:])
+    rows = sorted(int(r) for r in rows)
+    t0 = time.perf_counter()
+    ref = oracle.attn_varlen(t["q"], t["k"], t["v"], cu, cu, rows=rows)
+    cpu_s = time.perf_counter() - t0
+    got = outs[(args.steps - 1) % n_copies][rows].float().cpu().numpy().astype(np.float64)
+    diff = got - ref
+    max_abs = float(np.abs(diff).max())
+    rel = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+    seg_of = np.searchsorted(np.asarray(cu), np.asarray(rows), side="right") - 1
+    fl_rows = 4.0 * pw.D * pw.Hq * sum(float(lens[s]) for s in seg_of)
+    print(json.dumps({
+        "metric": METRIC + " (packed varlen segments)", "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": pw.name, "segments": pw.n_seg, "tokens": cu[-1], "min_len": min(lens),
+                   "max_len": max(lens), "heads_q": pw.Hq, "heads_kv": pw.Hkv, "head_dim": pw.D,
+                   "flop_per_step": fl, "l2": "inputs rotate over 4 device copies (> 126 MB L2)"},
+        "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                     "peak_kind": peak_kind, "traffic": None},
+        "oracle_check": {"max_abs": max_abs, "rel_l2": rel, "rows": f"{len(rows)} of {cu[-1]} x {pw.Hq} heads "
+                         "(first and last row of every segment + 96 seeded)", "bound": {"max_abs": 2e-2, "rel_l2": 1e-2},
+                         "pass": max_abs <= 2e-2 and rel <= 1e-2},
+        "cpu_baseline": {"value": fl_rows / cpu_s / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": f"{len(rows)} query rows x {pw.Hq} heads ({cpu_s:.1f} s)"},
+        "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
+    return 0
+
+
 def run_host(args, w):
     """Host cost of one call (validation, per-row metadata, five tensor-map
     encodings, launch) on the tiny workload, whose kernel is far shorter than
@@ -617,15 +697,20 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=list(workloads.WORKLOADS) + list(workloads.PACKED))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["attention", "prologue", "host"], default="attention",
                     help="prologue: time the optional fused Q/K RMSNorm+RoPE kernel instead; "
                          "host: host cost of one attention call (always the tiny workload)")
+    ap.add_argument("--exact", action="store_true",
+                    help="with --op prologue: time the bit-exact instance instead of the default fp32 one")
     ap.add_argument("--scatter", type=int, default=0,
                     help="N > 1: scatter the attention output over N destination buffers (fused all-to-all stores)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.workload in workloads.PACKED:
+        return run_packed(args, workloads.PACKED[args.workload])
     w = workloads.get(args.workload)
     if args.op == "prologue":
         return run_prologue(args, w)

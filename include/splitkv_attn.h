@@ -205,12 +205,24 @@ SK_API sk_status_t attn_fwd_varlen(const sk_tensor_t* q, const sk_tensor_t* k, c
  *   rope_table device fp32[table_rows, rot_dim] ([cos | sin]), table_rows >= S
  *   rot_dim    even, 0 <= rot_dim <= head_dim;  head_dim in {64, 128, 256}
  *   eps        >= 0
+ *   exact      0: evaluate the formula above in fp32 (sum of squares and
+ *              1/sqrt in fp32, both bf16 rounding points kept), bound by
+ *              memory bandwidth; each rotated result lies within three bf16
+ *              ulps, taken at the magnitude of its own two terms (|y_a*cs| +
+ *              |y_c*sn| for x_a, |y_c*cs| + |y_a*sn| for x_c), of the same
+ *              formula evaluated exactly with those two roundings (two for a
+ *              rare one-ulp difference in y carried through, one for the
+ *              final roundings); dims past rot_dim within one ulp of y.
+ *              1: return exactly the bits of that exact evaluation (fp32 with
+ *              an error bound, elements the bound cannot decide redone in
+ *              fp64), about 2.5 times slower.
+ * Returns SK_OK, SK_ERR_INVALID_ARG, SK_ERR_UNSUPPORTED or SK_ERR_CUDA.
  */
 SK_API sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, const void* w_q,
                             const void* w_k, const float* rope_table, int32_t table_rows,
                             int32_t rot_dim, int32_t interleaved, float eps,
                             int32_t num_q_heads, int32_t num_kv_heads, int32_t batch,
-                            int32_t head_dim, void* stream);
+                            int32_t head_dim, int32_t exact, void* stream);
 
 /*
  * sk_shard_pad_copy — one rank's chunk of a tail-padded sequence shard

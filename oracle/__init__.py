@@ -159,7 +159,8 @@ def attn_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix,
 def attn_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int],
                 seqused_q: Optional[Sequence[int]] = None,
                 seqused_k: Optional[Sequence[int]] = None,
-                softmax_scale: Optional[float] = None) -> np.ndarray:
+                softmax_scale: Optional[float] = None,
+                rows: Optional[Sequence[int]] = None) -> np.ndarray:
     """Packed variable-length attention, fp64 ("vLLM-Omni performance
     patterns": packed samples described by cu_seqlens; "sglang PR 30107":
     varlen attention over [valid | pad] segments).  The definition is a
@@ -169,7 +170,9 @@ def attn_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int
     and segments without a valid key, give zeros; rows outside every segment
     are returned as zeros too.
 
-    q [Tq, Hq, D] (or [1, Tq, Hq, D]), k/v [Tk, Hkv, D]; returns float64 [Tq, Hq, D].
+    q [Tq, Hq, D] (or [1, Tq, Hq, D]), k/v [Tk, Hkv, D]; returns float64 [Tq, Hq, D],
+    or with ``rows`` only those query rows (sorted, duplicates dropped):
+    [len(rows), Hq, D].
     """
     import torch
 
@@ -179,7 +182,8 @@ def attn_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int
     q3, k3, v3 = as3(q), as3(k), as3(v)
     Tq, Hq, D = q3.shape
     n = len(cu_seqlens_q) - 1
-    out = np.zeros((Tq, Hq, D), dtype=np.float64)
+    want = None if rows is None else np.asarray(sorted(set(int(r) for r in rows)), dtype=np.int64)
+    out = np.zeros((Tq if want is None else len(want), Hq, D), dtype=np.float64)
     empty = k3[:0].unsqueeze(0)
     for i in range(n):
         q0, q1 = int(cu_seqlens_q[i]), int(cu_seqlens_q[i + 1])
@@ -188,10 +192,17 @@ def attn_varlen(q, k, v, cu_seqlens_q: Sequence[int], cu_seqlens_k: Sequence[int
             continue
         nk = (k1 - k0) if seqused_k is None else int(seqused_k[i])
         nq = (q1 - q0) if seqused_q is None else int(seqused_q[i])
+        if want is None:
+            local, dst = None, slice(q0, q1)
+        else:
+            sel = np.nonzero((want >= q0) & (want < q1))[0]
+            if sel.size == 0:
+                continue
+            local, dst = [int(r) - q0 for r in want[sel]], sel
         seg = attn_split_kv(q3[q0:q1].unsqueeze(0), empty, empty,
                             k3[k0:k1].unsqueeze(0), v3[k0:k1].unsqueeze(0),
-                            real_len=[nk], q_valid=[nq], softmax_scale=softmax_scale)
-        out[q0:q1] = seg[0]
+                            real_len=[nk], q_valid=[nq], softmax_scale=softmax_scale, rows=local)
+        out[dst] = seg[0]
     return out
 
 

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version(L):
-    assert sk.sk_abi_version() == 1
+    assert sk.sk_abi_version() == 2
 
 
 def _t(len_s, sb, ss, sh, ptr=FAKE):
@@ -150,13 +150,13 @@ def test_prologue_rejects_bad_args(L):
     w = FAKE + (2 << 24)
     tab = FAKE + (3 << 24)
     # odd rot_dim
-    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 95, 0, 1e-6, 2, 1, 1, 128, None) == INVALID
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 95, 0, 1e-6, 2, 1, 1, 128, 0, None) == INVALID
     # unsupported head_dim
-    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 64, 0, 1e-6, 2, 1, 1, 96, None) == UNSUPPORTED
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 64, 0, 1e-6, 2, 1, 1, 96, 0, None) == UNSUPPORTED
     # table shorter than the sequence
-    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 7, 96, 0, 1e-6, 2, 1, 1, 128, None) == INVALID
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 7, 96, 0, 1e-6, 2, 1, 1, 128, 0, None) == INVALID
     # half-split rotary width not a multiple of 16
-    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 72, 0, 1e-6, 2, 1, 1, 128, None) == UNSUPPORTED
+    assert L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, tab, 8, 72, 0, 1e-6, 2, 1, 1, 128, 0, None) == UNSUPPORTED
 
 
 def test_python_binding_raises_on_missing_library(monkeypatch, tmp_path):
@@ -364,7 +364,7 @@ def test_prologue_rejects_q_k_sharing_tokens(L):
         q = _t(S, S * stride_s, stride_s, D)
         k = _t(S, S * stride_s, stride_s, D, ptr=FAKE + 2 * k_off_elems)
         return L.qk_rmsnorm_rope(ctypes.byref(q), ctypes.byref(k), w, w, FAKE, S, 64, 0,
-                                 ctypes.c_float(1e-6), Hq, Hkv, 1, D, None)
+                                 ctypes.c_float(1e-6), Hq, Hkv, 1, D, 0, None)
     assert call(ss) == 1                  # k = q shifted by one token
     assert call(Hq * D, stride_s=(Hq + 1) * D) == 1  # k's heads spill into q's next token
     assert b"overlap" in L.sk_last_error()

@@ -87,3 +87,21 @@ def test_varlen_oracle_single_segment_is_plain_attention(oracle_mod):
     empty = k[:0].unsqueeze(0)
     ref = oracle_mod.attn_split_kv(q.unsqueeze(0), empty, empty, k.unsqueeze(0), v.unsqueeze(0))
     assert np.array_equal(got, ref[0])
+
+
+def test_row_sample_equals_the_full_result(oracle_mod):
+    """oracle.attn_varlen(rows=...) returns exactly the selected rows of the
+    full result (sorted, duplicates dropped), including rows of empty
+    segments and rows outside every segment (zeros)."""
+    import numpy as np
+    import torch
+
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(70, 3, 64, generator=g).to(torch.bfloat16)
+    k = torch.randn(90, 3, 64, generator=g).to(torch.bfloat16)
+    v = torch.randn(90, 3, 64, generator=g).to(torch.bfloat16)
+    cq, ck = [2, 20, 20, 60], [0, 25, 40, 90]
+    full = oracle_mod.attn_varlen(q, k, v, cq, ck, seqused_k=[25, 0, 31])
+    rows = [65, 3, 19, 20, 59, 0, 3]
+    sub = oracle_mod.attn_varlen(q, k, v, cq, ck, seqused_k=[25, 0, 31], rows=rows)
+    assert np.array_equal(sub, full[sorted(set(rows))])

@@ -1,12 +1,26 @@
-"""Parity of the fused Q/K RMSNorm + RoPE prologue kernel with the fp64 oracle.
+"""Parity of the fused Q/K RMSNorm + RoPE prologue kernels with the fp64 oracle.
 
-Bar: every output element within 1 bf16 ulp of the oracle and at least
-99.99% bit-identical on the ordinary cases, where the ulp allowance covers a
-sum-of-squares reduction order that differs from the oracle's sequential one
-(it only matters when the row's squares span more than fp64's precision).
-The special-value, multi-block and large cases demand every bit: the kernel
-decides each bf16 rounding either from an fp32 value whose error bound
-keeps it off the rounding midpoint or by recomputing the element in fp64.
+Exact instance (exact=True).  Bar: every output element within 1 bf16 ulp of
+the oracle and at least 99.99% bit-identical on the ordinary cases, where the
+ulp allowance covers a sum-of-squares reduction order that differs from the
+oracle's sequential one (it only matters when the row's squares span more
+than fp64's precision).  The special-value, multi-block and large cases
+demand every bit: the kernel decides each bf16 rounding either from an fp32
+value whose error bound keeps it off the rounding midpoint or by recomputing
+the element in fp64.
+
+Default fp32 instance (exact=False): the same formula and rounding points in
+fp32.  Bound, derived from the arithmetic: y = bf16(x * r * w) is computed
+from an fp32 value within a few fp32 ulps of the exact one, so it equals the
+oracle's y or sits one bf16 ulp away (when the exact value is that close to a
+rounding midpoint); one bf16 ulp is at most 2^-7 of the value.  A rotated
+output z = y * c + y' * s' (c the cosine, s' the signed sine, y' the pair's
+other element) then moves by at most 2^-7 (|y c| + |y' s'|) = 2^-7 m <=
+2 ulp_bf16(m), m = |y c| + |y' s'| (the magnitude of its own two terms), and
+each side rounds once more (half an ulp of z <= half an ulp of m each):
+|z_gpu - z_ref| <= 3 ulp_bf16(m).  Dims past rot_dim are y itself: within
+1 ulp of |y|.  The tests also require at least 99.9% of the elements to be
+bit-identical.
 """
 import numpy as np
 import pytest
@@ -65,7 +79,7 @@ def test_prologue_matches_oracle(sk, D, rot, inter):
                                    rot_dim=rot, interleaved=inter, eps=eps)
     qd, kd = q.cuda(), k.cuda()
     tabd = tab.cuda() if rot else torch.zeros(S, 8, device="cuda")
-    sk.qk_rmsnorm_rope(qd, kd, wq.cuda(), wk.cuda(), tabd, rot_dim=rot, interleaved=inter, eps=1e-6)
+    sk.qk_rmsnorm_rope(qd, kd, wq.cuda(), wk.cuda(), tabd, rot_dim=rot, interleaved=inter, eps=1e-6, exact=True)
     torch.cuda.synchronize()
     _ulp_check(qd.cpu().view(torch.int16).numpy().view(np.uint16), ref_q)
     _ulp_check(kd.cpu().view(torch.int16).numpy().view(np.uint16), ref_k)
@@ -79,7 +93,8 @@ def test_prologue_in_place_on_fused_qkv_view(sk):
     wk = torch.randn(D, generator=gen).to(torch.bfloat16)
     tab = _table(S, 96)
     d = qkv.cuda()
-    sk.qk_rmsnorm_rope(d[:, :, :Hq], d[:, :, Hq:Hq + Hkv], wq.cuda(), wk.cuda(), tab.cuda(), eps=1e-5)
+    sk.qk_rmsnorm_rope(d[:, :, :Hq], d[:, :, Hq:Hq + Hkv], wq.cuda(), wk.cuda(), tab.cuda(), eps=1e-5,
+                       exact=True)
     torch.cuda.synchronize()
     got = d.cpu()
     assert torch.equal(got[:, :, Hq + Hkv:], qkv[:, :, Hq + Hkv:])  # v untouched
@@ -94,14 +109,14 @@ def _bits(t):
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def _run_both(sk, q, k, wq, wk, tab, rot, inter, eps):
+def _run_both(sk, q, k, wq, wk, tab, rot, inter, eps, exact=True):
     S = q.shape[1]
     eps32 = float(np.float32(eps))
     ref_q = oracle.qk_rmsnorm_rope(q, wq, tab.numpy(), rot_dim=rot, interleaved=inter, eps=eps32)
     ref_k = oracle.qk_rmsnorm_rope(k, wk, tab.numpy(), rot_dim=rot, interleaved=inter, eps=eps32)
     qd, kd = q.cuda(), k.cuda()
     tabd = tab.cuda() if rot else torch.zeros(S, 8, device="cuda")
-    sk.qk_rmsnorm_rope(qd, kd, wq.cuda(), wk.cuda(), tabd, rot_dim=rot, interleaved=inter, eps=eps)
+    sk.qk_rmsnorm_rope(qd, kd, wq.cuda(), wk.cuda(), tabd, rot_dim=rot, interleaved=inter, eps=eps, exact=exact)
     torch.cuda.synchronize()
     return _bits(qd.cpu()), ref_q, _bits(kd.cpu()), ref_k
 
@@ -220,3 +235,115 @@ def test_prologue_odd_head_count_bit_exact(sk, Hq, Hkv, D):
     gq, rq, gk, rk = _run_both(sk, q, k, wq, wk, tab, rot, False, 1e-6)
     assert np.array_equal(gq, rq), np.argwhere(gq != rq)[:5]
     assert np.array_equal(gk, rk), np.argwhere(gk != rk)[:5]
+
+
+# ---------------------------------------------------------------- default fp32 instance
+
+
+def _f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _ulp_bf16(m):
+    """bf16 ulp at magnitude m (0 for m == 0): 2^(floor(log2 m) - 7)."""
+    m = np.asarray(m, dtype=np.float64)
+    e = np.floor(np.log2(np.where(m > 0, m, 1.0)))
+    return np.where(m > 0, np.exp2(e - 7), 0.0)
+
+
+def _fast_check(got_bits, x, w, tab, rot, inter, eps32, min_identical=0.999):
+    """The default instance against the oracle: |z_gpu - z_ref| <= 3 ulp_bf16(m)
+    on rotated dims, m the magnitude of the output's own two terms (|y_a c| +
+    |y_p s| for the first element of a pair, |y_p c| + |y_a s| for the
+    second; y = the oracle's normalised value, c / s the pair's table
+    entries), within 1 ulp of |y| past rot_dim; and at least min_identical of
+    the elements bit-identical."""
+    ref = oracle.qk_rmsnorm_rope(x, w, tab.numpy(), rot_dim=rot, interleaved=inter, eps=eps32)
+    y = _f64(oracle.qk_rmsnorm_rope(x, w, np.zeros((tab.shape[0], 0), np.float32), rot_dim=0, eps=eps32))
+    B, S, H, D = y.shape
+    m = np.abs(y).copy()
+    allow = _ulp_bf16(m)
+    if rot:
+        t = tab.numpy().astype(np.float64)[:S]
+        half = rot // 2
+        i = np.arange(half)
+        if inter:
+            a_idx, p_idx = 2 * i, 2 * i + 1
+        else:
+            a_idx, p_idx = i, i + half
+        c = t[:, i][None, :, None, :]
+        sn = t[:, half + i][None, :, None, :]
+        ya, yp = y[..., a_idx], y[..., p_idx]
+        m[..., a_idx] = np.abs(ya * c) + np.abs(yp * sn)
+        m[..., p_idx] = np.abs(yp * c) + np.abs(ya * sn)
+        allow = _ulp_bf16(m)
+        allow[..., a_idx] *= 3
+        allow[..., p_idx] *= 3
+    g, r = _f64(got_bits), _f64(ref)
+    both_nan = np.isnan(g) & np.isnan(r)
+    same_inf = np.isinf(g) & (g == r)
+    diff = np.where(both_nan | same_inf, 0.0, np.abs(g - r))
+    assert not np.any(np.isnan(diff)), "NaN where the oracle has a number (or the reverse)"
+    bad = diff > allow
+    assert not bad.any(), (np.argwhere(bad)[:5], diff[bad][:5], allow[bad][:5])
+    ident = float((got_bits == ref).mean())
+    assert ident >= min_identical, ident
+    return ident
+
+
+@pytest.mark.parametrize("D,rot,inter", [(128, 96, False), (128, 128, False), (128, 96, True),
+                                          (64, 64, False), (64, 32, True), (256, 128, False),
+                                          (128, 0, False)])
+def test_fast_prologue_within_bound(sk, D, rot, inter):
+    gen = torch.Generator().manual_seed(100 + D + rot + int(inter))
+    B, S, Hq, Hkv = 2, 333, 6, 2
+    q = (torch.randn(B, S, Hq, D, generator=gen) * 2).to(torch.bfloat16)
+    k = (torch.randn(B, S, Hkv, D, generator=gen) * 0.5).to(torch.bfloat16)
+    wq = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    tab = _table(S + 5, rot) if rot else torch.zeros(S, 0)
+    gq, _, gk, _ = _run_both(sk, q, k, wq, wk, tab, rot, inter, 1e-6, exact=False)
+    eps32 = float(np.float32(1e-6))
+    _fast_check(gq, q, wq, tab, rot, inter, eps32)
+    _fast_check(gk, k, wk, tab, rot, inter, eps32)
+
+
+@pytest.mark.parametrize("inter", [False, True])
+def test_fast_prologue_large_and_special_values(sk, inter):
+    """About 5M elements per call, plus zero, inf and NaN rows (eps > 0): the
+    fp32 instance stays within the bound and propagates inf/NaN as the oracle
+    does.  (With eps = 0, a row whose squares all underflow fp32 differs: its
+    fp32 sum is 0; the exact instance covers that case.)"""
+    gen = torch.Generator().manual_seed(7 + int(inter))
+    B, S, Hq, Hkv, D, rot = 1, 4096, 8, 2, 128, 128
+    q = torch.randn(B, S, Hq, D, generator=gen)
+    k = torch.randn(B, S, Hkv, D, generator=gen) * 30
+    q[0, 1, 2] = 0.0
+    q[0, 4, 4, 7] = float("inf")
+    k[0, 5, 1, 9] = float("nan")
+    k[0, 3, 0, :] = -0.0
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    wq = (1 + 0.3 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (0.7 + 0.3 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    tab = _table(S, rot, theta=1e6)
+    gq, _, gk, _ = _run_both(sk, q, k, wq, wk, tab, rot, inter, 1e-6, exact=False)
+    eps32 = float(np.float32(1e-6))
+    _fast_check(gq, q, wq, tab, rot, inter, eps32)
+    _fast_check(gk, k, wk, tab, rot, inter, eps32)
+
+
+def test_fast_prologue_fused_view_leaves_v_untouched(sk):
+    gen = torch.Generator().manual_seed(2)
+    B, S, Hq, Hkv, D = 1, 300, 8, 2, 128
+    qkv = torch.randn(B, S, Hq + 2 * Hkv, D, generator=gen).to(torch.bfloat16)
+    wq = torch.randn(D, generator=gen).to(torch.bfloat16)
+    wk = torch.randn(D, generator=gen).to(torch.bfloat16)
+    tab = _table(S, 96)
+    d = qkv.cuda()
+    sk.qk_rmsnorm_rope(d[:, :, :Hq], d[:, :, Hq:Hq + Hkv], wq.cuda(), wk.cuda(), tab.cuda(), eps=1e-5)
+    torch.cuda.synchronize()
+    got = d.cpu()
+    assert torch.equal(got[:, :, Hq + Hkv:], qkv[:, :, Hq + Hkv:])
+    eps = float(np.float32(1e-5))
+    _fast_check(_bits(got[:, :, :Hq]), qkv[:, :, :Hq].contiguous(), wq, tab, 96, False, eps)
+    _fast_check(_bits(got[:, :, Hq:Hq + Hkv]), qkv[:, :, Hq:Hq + Hkv].contiguous(), wk, tab, 96, False, eps)

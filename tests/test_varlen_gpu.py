@@ -1,9 +1,10 @@
 """Parity of the packed variable-length entry point (attn_fwd_varlen, through
 the C ABI) with the fp64 oracle: unequal segment lengths around the 128/256-row
-tile edges, GQA, both head dims, more segments than one launch takes, pad
-exclusion through seqused_q/k (bitwise invariance to pad contents, exact zero
-pad rows), rows outside every segment left untouched.  Same bar as the other
-parity tests: max-abs <= 2e-2, relative L2 <= 1e-2."""
+tile edges, GQA, both head dims, hundreds of segments in one launch (and more
+than one launch holds), pad exclusion through seqused_q/k (bitwise invariance
+to pad contents, including NaN/Inf in the rows that share a segment's last
+key tile; exact zero pad rows), rows outside every segment left untouched.
+Same bar as the other parity tests: max-abs <= 2e-2, relative L2 <= 1e-2."""
 import numpy as np
 import pytest
 import torch
@@ -125,3 +126,71 @@ def test_varlen_rejections_raise(sk):
         sk.attn_fwd_varlen(q, k, k, [0, 70], [0, 80])
     with pytest.raises(sk.SplitKVError):
         sk.attn_fwd_varlen(q, k, k, [0, 64], [0, 80], seqused_k=[81])
+
+
+def _kernel_launches(fn):
+    """Attention kernel launches made by fn(), counted by the CUDA profiler."""
+    from torch.profiler import ProfilerActivity, profile
+
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return sum(e.count for e in prof.key_averages() if "attn_fwd" in e.key)
+
+
+@pytest.mark.parametrize("seed, n, D, Hq, Hkv, lo, hi", [
+    (20, 64, 128, 4, 2, 1, 700),
+    (21, 300, 64, 2, 1, 1, 200),
+])
+def test_many_segments_one_launch(sk, seed, n, D, Hq, Hkv, lo, hi):
+    g = torch.Generator().manual_seed(seed)
+    q_lens = torch.randint(lo, hi + 1, (n,), generator=g).tolist()
+    k_lens = torch.randint(lo, hi + 1, (n,), generator=g).tolist()
+    q, k, v, cq, ck = _packed(seed, q_lens, k_lens, Hq, Hkv, D)
+    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty_like(dq)
+    launches = _kernel_launches(lambda: sk.attn_fwd_varlen(dq, dk, dv, cq, ck, out=out))
+    assert launches == 1, launches
+    rows = sorted(set(torch.randint(0, cq[-1], (400,), generator=g).tolist()) | set(cq[:-1]))
+    ref = oracle.attn_varlen(q, k, v, cq, ck, rows=rows)
+    _compare(out[rows].float().cpu().numpy(), ref, f"{n} segments")
+    assert sk.sk_device_status() == 0
+
+
+def test_more_segments_than_one_launch_holds(sk):
+    """1100 short segments: two launches (1024 segments each at most)."""
+    n = 1100
+    g = torch.Generator().manual_seed(33)
+    q_lens = torch.randint(1, 40, (n,), generator=g).tolist()
+    k_lens = torch.randint(1, 40, (n,), generator=g).tolist()
+    q, k, v, cq, ck = _packed(33, q_lens, k_lens, 2, 2, 64)
+    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty_like(dq)
+    launches = _kernel_launches(lambda: sk.attn_fwd_varlen(dq, dk, dv, cq, ck, out=out))
+    assert launches == 2, launches
+    _compare(out.float().cpu().numpy(), oracle.attn_varlen(q, k, v, cq, ck), "1100 segments")
+
+
+def test_nan_rows_sharing_the_last_key_tile(sk):
+    """Segments whose last key tile is partial, followed by pad rows (seqused_k)
+    full of NaN and Inf: the pad rows share the tile with valid keys but must
+    not reach any output (the PV product must not see 0 * NaN)."""
+    D, Hq, Hkv = 128, 2, 2
+    g = torch.Generator().manual_seed(44)
+    seg = [(300, 150, 137), (200, 257, 250), (129, 129, 1)]  # (q rows, key rows, valid keys)
+    cq, ck, uk = [0], [0], []
+    for lq, lk, nk in seg:
+        cq.append(cq[-1] + lq); ck.append(ck[-1] + lk); uk.append(nk)
+    q = torch.randn(cq[-1], Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(ck[-1], Hkv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(ck[-1], Hkv, D, generator=g).to(torch.bfloat16)
+    ref = oracle.attn_varlen(q, k, v, cq, ck, seqused_k=uk)
+    for i, (lq, lk, nk) in enumerate(seg):
+        k[ck[i] + nk:ck[i + 1]] = float("nan")
+        v[ck[i] + nk:ck[i + 1]] = float("inf") if i % 2 else float("nan")
+    out = sk.attn_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), cq, ck, seqused_k=uk)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    _compare(got, ref, "NaN/Inf pad keys in the last tile")
+    assert sk.sk_device_status() == 0

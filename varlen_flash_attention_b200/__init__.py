@@ -92,7 +92,7 @@ def lib() -> ctypes.CDLL:
             L.attn_fwd_varlen.argtypes = [P, P, P, vp, vp, vp, vp, i32, i32, i32, ctypes.c_float, P, i32, vp]
             L.attn_fwd_varlen.restype = i32
             L.qk_rmsnorm_rope.argtypes = [P, P, vp, vp, vp, i32, i32, i32, ctypes.c_float, i32, i32,
-                                          i32, i32, vp]
+                                          i32, i32, i32, vp]
             L.qk_rmsnorm_rope.restype = i32
             L.sk_last_error.argtypes = []
             L.sk_last_error.restype = ctypes.c_char_p
@@ -401,11 +401,14 @@ def sk_shard_pad_copy(src, dst, first_row: int, pad_mode: str = "zeros", stream=
 
 
 def qk_rmsnorm_rope(q, k, w_q, w_k, rope_table, rot_dim: Optional[int] = None,
-                    interleaved: bool = False, eps: float = 1e-6, stream=None):
+                    interleaved: bool = False, eps: float = 1e-6, stream=None, exact: bool = False):
     """In-place fused RMSNorm(head_dim) + RoPE on q [B,S,Hq,D] and k [B,S,Hkv,D] (bf16, CUDA).
 
     rope_table: fp32 CUDA [rows >= S, rot_dim] holding [cos | sin] (its width
     is rot_dim); w_q, w_k: bf16 [D].  Every tensor on q's device.
+    exact: False (default) evaluates in fp32 (memory-bound, within one bf16
+    ulp of the exact result at the magnitude of the rotation's terms); True
+    returns the exact result's bits (slower).
     """
     import torch
 
@@ -436,7 +439,7 @@ def qk_rmsnorm_rope(q, k, w_q, w_k, rope_table, rot_dim: Optional[int] = None,
         st = lib().qk_rmsnorm_rope(ctypes.byref(dq), ctypes.byref(dk), w_q.data_ptr(), w_k.data_ptr(),
                                    rope_table.data_ptr() if rope_table.numel() else None,
                                    rope_table.shape[0], int(rot_dim), int(bool(interleaved)), float(eps),
-                                   Hq, Hkv, B, D, _stream_ptr(stream, dev))
+                                   Hq, Hkv, B, D, int(bool(exact)), _stream_ptr(stream, dev))
         _check(st)
     return q, k
 

@@ -84,6 +84,9 @@ struct alignas(64) AttnParams {
   // kernel publishes them).
   int32_t out_chunk;
   uint16_t* out_dst[kMaxOutDst];
+  int32_t n_heads;              // query heads (units: entry x head x row pair)
+  int32_t n_pairs;              // 256-row query blocks per entry (the longest entry's)
+  int32_t n_units;              // n_entries * n_heads * n_pairs
   int32_t group;                // num_q_heads / num_kv_heads
   float scale_log2;             // softmax_scale * log2(e)
   int32_t* status;              // device status word

@@ -71,6 +71,19 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- register budget
+// Move this warp's register allocation to N (multiple of 8, 24..256).  Every
+// warp of a warpgroup executes the same call; an increase waits until other
+// warps of the CTA have released enough with a decrease.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- tcgen05
 // TMEM allocation: executed by one full warp.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -106,6 +119,104 @@ __device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, u
       "elect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// As mma_ss_elect with the A operand (M x K, K-major) read from tensor memory
+// at column address a_tmem: 16-bit elements packed two per 32-bit column,
+// element k of a row in column k / 2 (low half for even k).
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// A whole 128 x N x (16 * KSTEPS) product as one instruction block: one
+// elect, then per K step only the descriptor offsets and the MMA, so the
+// issuing warp spends about three instructions per MMA (it shares its
+// sub-partition with busy softmax warps).  SS form: both operands in shared
+// memory, K-major, 128-byte swizzle, 64-column (128 B) sub-tiles kSubOff
+// (descriptor units of 16 B) apart; step k adds (k / 4) * kSubOff + (k % 4) * 2
+// to both start addresses (32 B per 16 elements inside a sub-tile).
+// accumulate == 0: the first step overwrites D.
+template <int KSTEPS, uint32_t kSubOff>
+__device__ __forceinline__ void mma_ss_block(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  static_assert(KSTEPS == 4 || KSTEPS == 8, "k steps");
+#define SKP_SS_STEP(K, ACC)                                                         \
+  "add.s64 ta, %1, " #K "; add.s64 tb, %2, " #K ";\n\t"                          \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, " ACC ";\n\t"
+  if constexpr (KSTEPS == 8) {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b64 ta, tb;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        SKP_SS_STEP(2, "1") SKP_SS_STEP(4, "1") SKP_SS_STEP(6, "1")
+        "add.s64 ta, %1, %5; add.s64 tb, %2, %5;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, 1;\n\t"
+        "add.s64 ta, %1, %6; add.s64 tb, %2, %6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, 1;\n\t"
+        "add.s64 ta, %1, %7; add.s64 tb, %2, %7;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, 1;\n\t"
+        "add.s64 ta, %1, %8; add.s64 tb, %2, %8;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ta, tb, %3, 1;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kSubOff), "n"(kSubOff + 2),
+        "n"(kSubOff + 4), "n"(kSubOff + 6)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b64 ta, tb;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        SKP_SS_STEP(2, "1") SKP_SS_STEP(4, "1") SKP_SS_STEP(6, "1") "}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+#undef SKP_SS_STEP
+}
+
+// TS form: A (M x K, K-major) in tensor memory at column a_tmem, 8 columns
+// per 16 elements of K; B (K x N, MN-major, 128-byte swizzle) in shared
+// memory, step k adds k * kBStep (descriptor units) to its start address.
+// Steps past ksteps (1..8) are not issued.
+template <uint32_t kBStep>
+__device__ __forceinline__ void mma_ts_block(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate, int ksteps) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, q, e_q;\n\t.reg .b64 tb;\n\t.reg .b32 ra;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "setp.gt.s32 q, %5, 1; and.pred e_q, e, q;\n\t"
+      "add.s32 ra, %1, 8; add.s64 tb, %2, %6;\n\t"
+      "@e_q tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], tb, %3, 1;\n\t"
+      "setp.gt.s32 q, %5, 2; and.pred e_q, e, q;\n\t"
+      "add.s32 ra, %1, 16; add.s64 tb, %2, %7;\n\t"
+      "@e_q tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], tb, %3, 1;\n\t"
+      "setp.gt.s32 q, %5, 3; and.pred e_q, e, q;\n\t"
+      "add.s32 ra, %1, 24; add.s64 tb, %2, %8;\n\t"
+      "@e_q tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], tb, %3, 1;\n\t"
+      "setp.gt.s32 q, %5, 4; and.pred e_q, e, q;\n\t"
+      "add.s32 ra, %1, 32; add.s64 tb, %2, %9;\n\t"
+      "@e_q tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], tb, %3, 1;\n\t"
+      "setp.gt.s32 q, %5, 5; and.pred e_q, e, q;\n\t"
+      "add.s32 ra, %1, 40; add.s64 tb, %2, %10;\n\t"
+      "@e_q tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], tb, %3, 1;\n\t"
+      "setp.gt.s32 q, %5, 6; and.pred e_q, e, q;\n\t"
+      "add.s32 ra, %1, 48; add.s64 tb, %2, %11;\n\t"
+      "@e_q tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], tb, %3, 1;\n\t"
+      "setp.gt.s32 q, %5, 7; and.pred e_q, e, q;\n\t"
+      "add.s32 ra, %1, 56; add.s64 tb, %2, %12;\n\t"
+      "@e_q tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], tb, %3, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(ksteps), "n"(kBStep), "n"(2 * kBStep),
+      "n"(3 * kBStep), "n"(4 * kBStep), "n"(5 * kBStep), "n"(6 * kBStep), "n"(7 * kBStep)
       : "memory");
 }
 
@@ -174,6 +285,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns; thread i of the warp writes lane (base lane + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // After tmem_wait_ld: tell the compiler the registers are (re)defined here, so no
 // use of them is scheduled above the wait.  Emits no instruction.
 template <int N>
@@ -215,6 +336,39 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pairs (one instruction for two lanes' worth of work): the pair
+// lives in one 64-bit register, .x in the low half.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -14,15 +14,18 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
+#include <cstddef>
 
 #include "../../include/splitkv_attn.h"
 #include "attn_fwd_sm100.cuh"
+#include "attn_fwd_persistent.cuh"
 #include "qk_norm_rope.cuh"
 #include "shard_copy.cuh"
 
 namespace {
 
-constexpr int32_t kAbiVersion = 1;
+constexpr int32_t kAbiVersion = 2;
 
 // ---------------------------------------------------------------- errors
 thread_local std::string g_last_error;
@@ -47,6 +50,9 @@ __device__ int32_t g_device_status = 0;
 
 uint64_t g_wait_limit_ns = 2000ull * 1000ull * 1000ull;
 int32_t g_test_stall = 0;
+// Attention kernel: 0 = persistent, P in TMEM, S(j+1) queued behind PV(j);
+// 1 = the same waiting for PV(j) to finish; 2 = one CTA per 256-row block.
+int32_t g_kernel_variant = 0;
 std::mutex g_mu;
 
 struct DeviceInfo {
@@ -54,7 +60,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sm_count = 0;
   int32_t* status = nullptr;
-  bool attn_attr_set[4] = {false, false, false, false};  // (D 64, D 128) x (plain, scattered)
+  bool attn_attr_set[40] = {};  // per kernel instance: cudaFuncSetAttribute done
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -103,8 +109,49 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // 3-D map over (d, head, seq) of one batch row: box = 64 d x 1 head x 128 rows,
 // 128-byte swizzle.  `rows` is the clipped sequence extent (>= 1).
+//
+// An encoded map is a pure function of its inputs (address, extents,
+// strides; type, box and swizzle are fixed here), so encoded maps are kept in
+// a small per-thread cache keyed on exactly those inputs: a caller that
+// passes the same buffers again (the caching allocator hands the same
+// addresses back every step) skips the driver's encoder.
+struct MapKey {
+  const void* base;
+  int64_t stride_s, stride_h, rows;
+  int32_t heads, D;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && stride_s == o.stride_s && stride_h == o.stride_h && rows == o.rows &&
+           heads == o.heads && D == o.D;
+  }
+};
+
+struct MapCache {
+  static constexpr int kWays = 64;
+  MapKey key[kWays];
+  CUtensorMap map[kWays];
+  uint32_t stamp[kWays] = {};
+  uint32_t clock = 0;
+  bool valid[kWays] = {};
+};
+thread_local MapCache g_map_cache;
+
 sk_status_t encode_map(CUtensorMap* m, const void* base, int64_t stride_s, int64_t stride_h,
                        int heads, int64_t rows, int D) {
+  const MapKey k{base, stride_s, stride_h, rows, heads, D};
+  MapCache& c = g_map_cache;
+  int victim = -1;  // an empty slot if there is one, else the least recently used
+  for (int i = 0; i < MapCache::kWays; ++i) {
+    if (!c.valid[i]) {
+      if (victim < 0 || c.valid[victim]) victim = i;
+      continue;
+    }
+    if (c.key[i] == k) {
+      c.stamp[i] = ++c.clock;
+      *m = c.map[i];
+      return SK_OK;
+    }
+    if (victim < 0 || (c.valid[victim] && c.stamp[i] < c.stamp[victim])) victim = i;
+  }
   auto enc = get_encode_fn();
   if (!enc) return fail(SK_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
@@ -116,6 +163,10 @@ sk_status_t encode_map(CUtensorMap* m, const void* base, int64_t stride_s, int64
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  c.key[victim] = k;
+  c.map[victim] = *m;
+  c.valid[victim] = true;
+  c.stamp[victim] = ++c.clock;
   return SK_OK;
 }
 
@@ -182,21 +233,63 @@ sk_status_t check_tensor(const char* name, const sk_tensor_t* t, int B, int H, i
 }
 
 template <int D>
-sk_status_t launch_attn(const skattn::AttnParams& prm, int n_qtiles, int H, int nb, cudaStream_t stream,
-                        DeviceInfo* dev) {
-  using L = skattn::SmemLayout<D>;
-  const bool scatter = prm.out_chunk > 0;  // separate instance: the plain kernel's code is untouched
-  const int slot = (D == 64 ? 0 : 1) + (scatter ? 2 : 0);
-  auto kernel = scatter ? skattn::attn_fwd_kernel<D, true> : skattn::attn_fwd_kernel<D, false>;
+sk_status_t set_smem(const void* kernel, int slot, uint32_t bytes, DeviceInfo* dev, int launch_regs = 0) {
   if (!dev->attn_attr_set[slot]) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (launch_regs > 0) {
+      // The kernel moves registers between its warpgroups (setmaxnreg); that
+      // split adds up only if it is launched with exactly this many.
+      cudaFuncAttributes a;
+      cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+      if (a.numRegs != launch_regs)
+        return fail(SK_ERR_UNSUPPORTED, "attention kernel built with %d registers per thread, %d expected",
+                    a.numRegs, launch_regs);
+    }
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     dev->attn_attr_set[slot] = true;
   }
-  dim3 grid(n_qtiles, H, nb);
-  kernel<<<grid, skattn::kThreads, L::kAlloc, stream>>>(prm);
+  return SK_OK;
+}
+
+template <int D>
+sk_status_t launch_attn(skattn::AttnParams& prm, int n_qtiles, int H, int nb, cudaStream_t stream,
+                        DeviceInfo* dev) {
+  const bool scatter = prm.out_chunk > 0;  // separate instance: the plain kernel's code is untouched
+  const int variant = g_kernel_variant;
+  const int slot = (D == 64 ? 0 : 1) + (scatter ? 2 : 0) + 4 * variant;  // 0..23
+  sk_status_t st;
+  if (variant == 2) {
+    using L = skattn::SmemLayout<D>;
+    auto kernel = scatter ? skattn::attn_fwd_kernel<D, true> : skattn::attn_fwd_kernel<D, false>;
+    if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev)) != SK_OK) return st;
+    dim3 grid(n_qtiles, H, nb);
+    kernel<<<grid, skattn::kThreads, L::kAlloc, stream>>>(prm);
+  } else {
+    using L = skattn::PSmemLayout<D>;
+    using P = skattn::AttnParams;
+    void (*kernel)(P) = nullptr;
+    switch (variant) {
+      case 1: kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, true, 0, P>
+                               : skattn::attn_fwd_persistent_kernel<D, false, true, 0, P>; break;
+      case 3: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 2, P>; break;
+      case 4: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 3, P>; break;
+      case 5: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 4, P>; break;
+      default: kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, false, 0, P>
+                                : skattn::attn_fwd_persistent_kernel<D, false, false, 0, P>; break;
+    }
+    if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev, skattn::kLaunchRegs)) != SK_OK)
+      return st;
+    prm.n_heads = H;
+    prm.n_pairs = n_qtiles;
+    const int64_t units = static_cast<int64_t>(nb) * H * n_qtiles;
+    if (units > INT32_MAX) return fail(SK_ERR_UNSUPPORTED, "too many work units (%lld)", (long long)units);
+    prm.n_units = static_cast<int32_t>(units);
+    const int grid = static_cast<int>(std::min<int64_t>(units, dev->sm_count));
+    kernel<<<grid, skattn::kPThreads, L::kAlloc, stream>>>(prm);
+  }
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
   return SK_OK;
 }
 
@@ -333,6 +426,91 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
   return SK_OK;
 }
 
+// Packed varlen input on the persistent kernel: one tensor map per packed
+// tensor, the segments' rows and lengths in the launch parameters, segments
+// processed longest first (a static schedule over the SMs balances best when
+// the big units come first); one launch per kMaxSegments segments.
+template <int D>
+sk_status_t launch_varlen(skattn::VarlenParams& prm, cudaStream_t stream, DeviceInfo* dev) {
+  using L = skattn::PSmemLayout<D>;
+  const int variant = g_kernel_variant;
+  const int slot = 24 + (D == 64 ? 0 : 1) + 2 * (variant == 1);  // 24..27
+  auto kernel = variant == 1 ? skattn::attn_fwd_persistent_kernel<D, false, true, 0, skattn::VarlenParams>
+                             : skattn::attn_fwd_persistent_kernel<D, false, false, 0, skattn::VarlenParams>;
+  sk_status_t st;
+  if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev, skattn::kLaunchRegs)) != SK_OK)
+    return st;
+  const int grid = std::min(prm.n_units, dev->sm_count);
+  kernel<<<grid, skattn::kPThreads, L::kAlloc, stream>>>(prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch (packed)");
+  return SK_OK;
+}
+
+sk_status_t varlen_persistent(const sk_tensor_t* q, const sk_tensor_t* k, const sk_tensor_t* v,
+                              const int32_t* cu_q, const int32_t* cu_k, const int32_t* used_q,
+                              const int32_t* used_k, int32_t nseg, int32_t Hq, int32_t Hkv, float scale,
+                              const sk_tensor_t* out, int32_t D, cudaStream_t stream, DeviceInfo* info) {
+  struct Seg { int32_t q0, k0, lq, qv, nk; int64_t cost; };
+  std::vector<Seg> segs;
+  segs.reserve(nseg);
+  bool any_q = false, any_k = false;
+  for (int i = 0; i < nseg; ++i) {
+    Seg g;
+    g.q0 = cu_q[i];
+    g.k0 = cu_k[i];
+    g.lq = cu_q[i + 1] - cu_q[i];
+    g.qv = used_q ? used_q[i] : g.lq;
+    g.nk = used_k ? used_k[i] : cu_k[i + 1] - cu_k[i];
+    if (g.lq == 0) continue;  // no rows: nothing to write
+    const int64_t pairs = (g.lq + skattn::kRowsPerCta - 1) / skattn::kRowsPerCta;
+    const int64_t tiles = (g.nk + skattn::kBlockN - 1) / skattn::kBlockN;
+    g.cost = pairs * std::max<int64_t>(tiles, 1);
+    any_q = any_q || (g.qv > 0 && g.nk > 0);
+    any_k = any_k || g.nk > 0;
+    segs.push_back(g);
+  }
+  std::stable_sort(segs.begin(), segs.end(), [](const Seg& a, const Seg& b) { return a.cost > b.cost; });
+  static thread_local skattn::VarlenParams prm;
+  std::memset(static_cast<void*>(&prm), 0, offsetof(skattn::VarlenParams, seg_unit0));
+  sk_status_t st;
+  if (any_q && any_k) {
+    if ((st = encode_map(&prm.tm_q, q->ptr, q->stride_s, q->stride_h, Hq, q->len_s, D)) != SK_OK) return st;
+    if ((st = encode_map(&prm.tm_k, k->ptr, k->stride_s, k->stride_h, Hkv, k->len_s, D)) != SK_OK) return st;
+    if ((st = encode_map(&prm.tm_v, v->ptr, v->stride_s, v->stride_h, Hkv, v->len_s, D)) != SK_OK) return st;
+  }
+  prm.out = static_cast<uint16_t*>(out->ptr);
+  prm.out_ss = out->stride_s;
+  prm.out_sh = out->stride_h;
+  prm.n_heads = Hq;
+  prm.group = Hq / Hkv;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.status = info->status;
+  prm.wait_limit_ns = g_wait_limit_ns;
+  prm.test_stall = g_test_stall;
+  for (size_t s0 = 0; s0 < segs.size(); s0 += skattn::kMaxSegments) {
+    const int n = static_cast<int>(std::min<size_t>(skattn::kMaxSegments, segs.size() - s0));
+    int64_t units = 0;
+    for (int i = 0; i < n; ++i) {
+      const Seg& g = segs[s0 + i];
+      if (units > INT32_MAX) return fail(SK_ERR_UNSUPPORTED, "too many work units");
+      prm.seg_unit0[i] = static_cast<int32_t>(units);
+      prm.seg_q0[i] = g.q0;
+      prm.seg_k0[i] = g.k0;
+      prm.seg_lq[i] = g.lq;
+      prm.seg_qv[i] = g.qv;
+      prm.seg_nk[i] = g.nk;
+      units += static_cast<int64_t>(Hq) * ((g.lq + skattn::kRowsPerCta - 1) / skattn::kRowsPerCta);
+    }
+    if (units > INT32_MAX) return fail(SK_ERR_UNSUPPORTED, "too many work units");
+    prm.n_seg = n;
+    prm.n_units = static_cast<int32_t>(units);
+    st = (D == 64) ? launch_varlen<64>(prm, stream, info) : launch_varlen<128>(prm, stream, info);
+    if (st != SK_OK) return st;
+  }
+  return SK_OK;
+}
+
 // Packed varlen input: segment i owns query rows [cu_q[i], cu_q[i+1]) and key
 // rows [cu_k[i], cu_k[i+1]) of single-row tensors; each segment becomes one
 // kernel entry whose tensor maps start at the segment's first row (no prefix,
@@ -384,6 +562,8 @@ sk_status_t varlen_impl(const sk_tensor_t* q, const sk_tensor_t* k, const sk_ten
   DeviceInfo* info = nullptr;
   if ((st = device_setup(&dev, &info)) != SK_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  if (g_kernel_variant != 2)
+    return varlen_persistent(q, k, v, cu_q, cu_k, used_q, used_k, nseg, Hq, Hkv, scale, out, D, stream, info);
   auto rptr = [](const sk_tensor_t* t, int64_t row) {
     return static_cast<const void*>(static_cast<const uint16_t*>(t->ptr) + row * t->stride_s);
   };
@@ -546,7 +726,7 @@ sk_status_t sk_shard_pad_copy(const void* src, int64_t src_stride_b, int64_t src
 sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, const void* w_q, const void* w_k,
                             const float* rope_table, int32_t table_rows, int32_t rot_dim,
                             int32_t interleaved, float eps, int32_t num_q_heads, int32_t num_kv_heads,
-                            int32_t batch, int32_t head_dim, void* stream) {
+                            int32_t batch, int32_t head_dim, int32_t exact, void* stream) {
   try {
     if (batch < 0) return fail(SK_ERR_INVALID_ARG, "batch < 0");
     if (num_q_heads <= 0 || num_kv_heads <= 0) return fail(SK_ERR_INVALID_ARG, "head counts must be positive");
@@ -608,7 +788,7 @@ sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, const vo
     prm.Hq = num_q_heads;
     prm.Hkv = num_kv_heads;
     prm.B = batch;
-    cudaError_t e = skqkn::launch(prm, head_dim, static_cast<cudaStream_t>(stream));
+    cudaError_t e = skqkn::launch(prm, head_dim, exact != 0, info->sm_count, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "qk_rmsnorm_rope launch");
     return SK_OK;
   } catch (...) {
@@ -652,6 +832,21 @@ sk_status_t sk_test_stall_mma(int32_t on) {
 }
 
 int32_t sk_abi_version(void) { return kAbiVersion; }
+
+SK_API sk_status_t sk_debug_prologue_variant(int32_t v) {
+  if (v < 0 || v > 4) return fail(SK_ERR_INVALID_ARG, "variant must be in 0..4");
+  skqkn::fast_variant() = v;
+  return SK_OK;
+}
+
+// Development hook (not part of the header's interface): selects the
+// attention kernel variant for side-by-side timing.
+SK_API sk_status_t sk_debug_kernel_variant(int32_t v) {
+  if (v < 0 || v > 5) return fail(SK_ERR_INVALID_ARG, "variant must be in 0..5");
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_kernel_variant = v;
+  return SK_OK;
+}
 
 
 }  // extern "C"

@@ -32,6 +32,9 @@ __all__ = [
     "make_inputs",
     "poison_pad",
     "random_workload",
+    "PackedWorkload",
+    "PACKED",
+    "make_packed",
 ]
 
 
@@ -179,3 +182,51 @@ def random_workload(
     seed = ri(0, 2**31 - 1)
     return Workload(name, B=B, Hq=Hq, Hkv=Hkv, D=D, Sq=Sq, Sp=Sp, Ss=Ss,
                     real_len=real_len, seed=seed)
+
+
+@dataclasses.dataclass(frozen=True)
+class PackedWorkload:
+    """Packed variable-length self-attention: ``n_seg`` independent samples of
+    lengths drawn uniformly from [min_len, max_len] (a CPU generator seeded
+    with ``seed``), concatenated on one token axis (cu_seqlens)."""
+
+    name: str
+    n_seg: int
+    min_len: int
+    max_len: int
+    Hq: int
+    Hkv: int
+    D: int
+    seed: int
+    description: str = ""
+
+
+PACKED: Dict[str, PackedWorkload] = {
+    w.name: w
+    for w in [
+        PackedWorkload(
+            "packed", n_seg=64, min_len=256, max_len=4096, Hq=16, Hkv=16, D=128, seed=7,
+            description="64 packed samples of 256-4096 tokens (image/video latents of mixed "
+                        "resolutions in one batch), self-attention within each sample",
+        ),
+    ]
+}
+
+
+def make_packed(w: PackedWorkload) -> Dict[str, object]:
+    """Draw the segment lengths, then q [T, Hq, D], k and v [T, Hkv, D] (bf16,
+    N(0,1)) in that order from one generator; cu_seqlens shared by q and k."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(w.seed)
+    lens = torch.randint(w.min_len, w.max_len + 1, (w.n_seg,), generator=gen).tolist()
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + int(n))
+    T = cu[-1]
+    return {
+        "q": _draw(gen, (T, w.Hq, w.D), 1.0),
+        "k": _draw(gen, (T, w.Hkv, w.D), 1.0),
+        "v": _draw(gen, (T, w.Hkv, w.D), 1.0),
+        "cu_seqlens": cu,
+        "lens": [int(n) for n in lens],
+    }
