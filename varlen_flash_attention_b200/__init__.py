@@ -108,6 +108,28 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
+_fast = None
+
+
+def _fastcall():
+    """The compiled marshalling module for attn_fwd_split_kv (built in-tree by
+    build.build_binding; raises if it cannot be built or loaded)."""
+    global _fast
+    if _fast is None:
+        with _lock:
+            if _fast is None:
+                if not os.path.exists(LIB_PATH):
+                    raise ImportError(
+                        f"{LIB_PATH} is missing: build it with "
+                        "`python -m varlen_flash_attention_b200.build` (nvcc, sm_100a)")
+                from . import build as _build
+
+                m = _build.build_binding()
+                m.bind_library(LIB_PATH)
+                _fast = m
+    return _fast
+
+
 def _check(status: int) -> None:
     if status != 0:
         msg = lib().sk_last_error()
@@ -231,34 +253,28 @@ def attn_fwd_split_kv(q, k_prefix, v_prefix, k_suffix, v_suffix,
     kernel gave up a bounded wait (otherwise such a failure is only visible
     through sk_device_status).  Returns ``out`` ([B, Sq, Hq, D] bf16,
     allocated if not given).
+
+    The checks and the descriptors are built by a small compiled module
+    (argument marshalling only), which keeps the host cost of a call close to
+    the C ABI's own.
     """
     import torch
 
-    kv = (("k_prefix", k_prefix), ("v_prefix", v_prefix), ("k_suffix", k_suffix), ("v_suffix", v_suffix))
-    Hkv = _check_attn_shapes(q, kv, out)
-    B, Sq, Hq, D = q.shape
-    dev = q.device
-    _same_device(dev, kv + (("out", out),))
     if out is None:
-        out = torch.empty((B, Sq, Hq, D), dtype=q.dtype, device=dev)
+        if q.dim() != 4:
+            raise ValueError("q must be [batch, seq, heads, head_dim]")
+        out = torch.empty(tuple(q.shape), dtype=q.dtype, device=q.device)
     if softmax_scale is None:
-        softmax_scale = D ** -0.5
-    descs = [tensor_desc(t) for t in (q, k_prefix, v_prefix, k_suffix, v_suffix, out)]
-    rl = _int32_array(real_len, B)
-    qv = _int32_array(q_valid, B)
-    L = lib()
-    args = [ctypes.byref(d) for d in descs[:5]] + [
-        ctypes.cast(rl, ctypes.c_void_p) if rl is not None else None, Hq, Hkv, float(softmax_scale),
-        ctypes.byref(descs[5]), B, D]
-    with _OnDevice(dev):
-        sp = _stream_ptr(stream, dev)
-        if qv is None:
-            st = L.attn_fwd_split_kv(*args, sp)
-        else:
-            st = L.attn_fwd_split_kv_ex(*args, ctypes.cast(qv, ctypes.c_void_p), sp)
+        softmax_scale = q.shape[-1] ** -0.5
+    sp = 0 if stream is None else (stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    st = _fastcall().attn_fwd_split_kv(
+        q, k_prefix, v_prefix, k_suffix, v_suffix, out,
+        None if real_len is None else [int(v) for v in real_len],
+        None if q_valid is None else [int(v) for v in q_valid], float(softmax_scale), sp)
+    if st:
         _check(st)
-        if check_status:
-            _raise_if_device_timeout(dev)
+    if check_status:
+        _raise_if_device_timeout(q.device)
     return out
 
 

@@ -40,6 +40,21 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
+BINDING_SRC = os.path.join(HERE, "csrc", "binding.cpp")
+EXT_DIR = os.path.join(HERE, "_build", "skfast")
+EXT_NAME = "skfast"
+
+
+def build_binding(verbose: bool = False):
+    """Compile (or load, when up to date) the compiled argument-marshalling
+    module for attn_fwd_split_kv, in-tree under _build/skfast; returns it."""
+    from torch.utils.cpp_extension import load
+
+    os.makedirs(EXT_DIR, exist_ok=True)
+    return load(name=EXT_NAME, sources=[BINDING_SRC], build_directory=EXT_DIR,
+                extra_cflags=["-O2", "-I" + os.path.join(ROOT, "include")], with_cuda=True, verbose=verbose)
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if not force and up_to_date():
         return LIB_PATH
@@ -53,3 +68,4 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv))
+    print(build_binding().__file__)

@@ -8,7 +8,7 @@
 // rotation partner (d + rot_dim/2) lives rot_dim/16 lanes away and is fetched
 // with one shuffle of the already bf16-rounded normalised values.
 //
-// Two instances.  The default (qk_norm_rope_fast_kernel) evaluates the
+// Two instances.  The default (qk_norm_rope_warp_kernel) evaluates the
 // unfused path in fp32 with its two bf16 rounding points: the sum of squares
 // and r = rsqrt(mean + eps) in fp32, y = bf16(x * r * w), then the rotation
 // z = bf16(y * cos -/+ y_partner * sin) with one fused multiply-add; about ten
@@ -353,154 +353,7 @@ __global__ void __launch_bounds__(kNormRopeThreads, kNormRopeMinBlocks) qk_norm_
   }
 }
 
-// fp32 instance: D/8 lanes per token walk the token's rows four at a time
-// with the next four already in flight (8 x 16 bytes outstanding per lane:
-// enough bytes in flight to cover HBM latency at two blocks per SM), blocks
-// striding over the tokens so the grid is one resident wave; no fp64 and no
-// fix-ups.
 constexpr int kFastThreads = 256;
-
-template <int D, int BATCH, int MINB>
-__global__ void __launch_bounds__(kFastThreads, MINB) qk_norm_rope_fast_kernel(const NormRopeParams p) {
-  constexpr int TPR = D / 8;                   // lanes per row
-  constexpr int GROUPS = kFastThreads / TPR;   // tokens per block and pass
-  __shared__ __align__(16) float w_s[2][D];
-  for (int i = threadIdx.x; i < 2 * D; i += blockDim.x)
-    w_s[i / D][i % D] = __uint_as_float(static_cast<uint32_t>((i < D ? p.w_q : p.w_k)[i % D]) << 16);
-  __syncthreads();
-
-  const int sub = threadIdx.x % TPR;
-  const int lane = threadIdx.x % 32;
-  const int d0 = sub * 8;
-  const int rot = p.rot_dim;
-  const bool rotates = d0 < rot;
-  int src = lane;
-  if (!p.interleaved && rot > 0) {
-    const int half = rot / 2, hs = half / 8;
-    if (d0 < half) src = lane + hs;
-    else if (d0 < rot) src = lane - hs;
-  }
-  const int H = p.Hq + p.Hkv;
-  const float inv_d = 1.0f / static_cast<float>(D);
-  const int64_t n_tok = static_cast<int64_t>(p.B) * p.S;
-  // every lane of a warp runs the same number of passes (shuffles stay full-warp)
-  const int64_t passes = (n_tok + static_cast<int64_t>(gridDim.x) * GROUPS - 1) / (static_cast<int64_t>(gridDim.x) * GROUPS);
-
-  for (int64_t pass = 0; pass < passes; ++pass) {
-    const int64_t tok = (pass * gridDim.x + blockIdx.x) * GROUPS + threadIdx.x / TPR;
-    const bool valid = tok < n_tok;
-    const int s = valid ? static_cast<int>(tok % p.S) : 0;
-    const int b = valid ? static_cast<int>(tok / p.S) : 0;
-
-    float c[8], sg[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { c[i] = 1.0f; sg[i] = 0.0f; }
-    if (rotates && valid) {
-      const float* crow = p.table + static_cast<int64_t>(s) * rot;
-      if (p.interleaved) {
-        const float4 c4 = *reinterpret_cast<const float4*>(crow + d0 / 2);
-        const float4 s4 = *reinterpret_cast<const float4*>(crow + rot / 2 + d0 / 2);
-        const float cv[4] = {c4.x, c4.y, c4.z, c4.w};
-        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          c[2 * e] = c[2 * e + 1] = cv[e];
-          sg[2 * e] = -sv[e];
-          sg[2 * e + 1] = sv[e];
-        }
-      } else {
-        const int half = rot / 2;
-        const bool first = d0 < half;
-        const int i0 = first ? d0 : d0 - half;
-        const float4 c0 = *reinterpret_cast<const float4*>(crow + i0);
-        const float4 c1 = *reinterpret_cast<const float4*>(crow + i0 + 4);
-        const float4 s0 = *reinterpret_cast<const float4*>(crow + half + i0);
-        const float4 s1 = *reinterpret_cast<const float4*>(crow + half + i0 + 4);
-        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          c[e] = cv[e];
-          sg[e] = first ? -sv[e] : sv[e];
-        }
-      }
-    }
-    uint16_t* qrow = p.q + b * p.q_sb + s * p.q_ss + d0;
-    uint16_t* krow = p.k + b * p.k_sb + s * p.k_ss + d0 - static_cast<int64_t>(p.Hq) * p.k_sh;
-    auto row_ptr = [&](int h) { return h < p.Hq ? qrow + h * p.q_sh : krow + h * p.k_sh; };
-
-    uint4 xv[BATCH];
-#pragma unroll
-    for (int j = 0; j < BATCH; ++j)
-      xv[j] = (valid && j < H) ? *reinterpret_cast<const uint4*>(row_ptr(j)) : make_uint4(0, 0, 0, 0);
-
-    for (int h0 = 0; h0 < H; h0 += BATCH) {
-      uint4 xn[BATCH];
-#pragma unroll
-      for (int j = 0; j < BATCH; ++j) {
-        const int h = h0 + BATCH + j;
-        xn[j] = (valid && h < H) ? *reinterpret_cast<const uint4*>(row_ptr(h)) : make_uint4(0, 0, 0, 0);
-      }
-      float ss[BATCH];
-#pragma unroll
-      for (int j = 0; j < BATCH; ++j) {
-        const uint32_t xw[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
-        float a = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float lo = bf16_lo(xw[i]), hi = bf16_hi(xw[i]);
-          a = fmaf(lo, lo, a);
-          a = fmaf(hi, hi, a);
-        }
-        ss[j] = a;
-      }
-#pragma unroll
-      for (int o = TPR / 2; o > 0; o >>= 1) {
-#pragma unroll
-        for (int j = 0; j < BATCH; ++j) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], o);
-      }
-#pragma unroll
-      for (int j = 0; j < BATCH; ++j) {
-        const int h = h0 + j;
-        if (h >= H) break;
-        const float r = rsqrtf(fmaf(ss[j], inv_d, p.eps));
-        const float* w = w_s[h < p.Hq ? 0 : 1] + d0;
-        const float4 w0 = *reinterpret_cast<const float4*>(w);
-        const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        const uint32_t xw[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
-        uint32_t yb[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          yb[i] = pack_bf16x2_rn(bf16_lo(xw[i]) * r * wv[2 * i], bf16_hi(xw[i]) * r * wv[2 * i + 1]);
-        uint32_t pb[4];
-        if (p.interleaved) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) pb[i] = __byte_perm(yb[i], 0, 0x1032);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) pb[i] = __shfl_sync(0xffffffffu, yb[i], src);
-        }
-        uint32_t zb[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float za = fmaf(bf16_lo(pb[i]), sg[2 * i], bf16_lo(yb[i]) * c[2 * i]);
-          const float zc = fmaf(bf16_hi(pb[i]), sg[2 * i + 1], bf16_hi(yb[i]) * c[2 * i + 1]);
-          zb[i] = rotates ? pack_bf16x2_rn(za, zc) : yb[i];
-        }
-        if (valid) *reinterpret_cast<uint4*>(row_ptr(h)) = make_uint4(zb[0], zb[1], zb[2], zb[3]);
-      }
-#pragma unroll
-      for (int j = 0; j < BATCH; ++j) xv[j] = xn[j];
-    }
-  }
-}
-
-// Development hook: launch shape of the fp32 instance (0 = shipped).
-inline int& fast_variant() {
-  static int v = 0;
-  return v;
-}
 
 // fp32 instance, one token per warp: 32 / (D/8) rows per load instruction,
 // so a warp streams through its token's heads in contiguous runs (BATCH
@@ -637,7 +490,7 @@ __global__ void __launch_bounds__(kFastThreads, MINB) qk_norm_rope_warp_kernel(c
   }
 }
 
-inline cudaError_t launch(const NormRopeParams& p, int D, bool exact, int sm_count, cudaStream_t stream) {
+inline cudaError_t launch(const NormRopeParams& p, int D, bool exact, cudaStream_t stream) {
   const int64_t tokens = static_cast<int64_t>(p.B) * p.S;
   const int groups = kNormRopeThreads / (D / 8);
   const int64_t blocks = (tokens + groups - 1) / groups;
@@ -652,29 +505,14 @@ inline cudaError_t launch(const NormRopeParams& p, int D, bool exact, int sm_cou
       default: return cudaErrorInvalidValue;
     }
   } else {
-    // blocks stride over the tokens; `waves` resident waves of MINB blocks per SM
-    const int64_t per_block = kFastThreads / (D / 8);
-    const int64_t need = (tokens + per_block - 1) / per_block;
-    auto go = [&](auto kern, int minb, int waves) {
-      const unsigned gf = static_cast<unsigned>(std::min<int64_t>(need, static_cast<int64_t>(sm_count) * minb * waves));
-      kern<<<gf, kFastThreads, 0, stream>>>(p);
-    };
-    const int v = fast_variant();
+    // one token per warp, kFastThreads / 32 tokens per block
+    const int64_t wblocks = (tokens + kFastThreads / 32 - 1) / (kFastThreads / 32);
+    if (wblocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const unsigned gw = static_cast<unsigned>(wblocks);
     switch (D) {
-      case 64: go(qk_norm_rope_fast_kernel<64, 2, 3>, 3, 64); break;
-      case 128:
-        if (v == 1 || v == 2 || v == 3) {
-          const unsigned gw = static_cast<unsigned>((tokens + kFastThreads / 32 - 1) / (kFastThreads / 32));
-          if (v == 1) qk_norm_rope_warp_kernel<128, 2, 3><<<gw, kFastThreads, 0, stream>>>(p);
-          else if (v == 2) qk_norm_rope_warp_kernel<128, 4, 2><<<gw, kFastThreads, 0, stream>>>(p);
-          else qk_norm_rope_warp_kernel<128, 1, 4><<<gw, kFastThreads, 0, stream>>>(p);
-        } else if (v == 4) {
-          go(qk_norm_rope_fast_kernel<128, 4, 2>, 2, 1);
-        } else {
-          go(qk_norm_rope_fast_kernel<128, 2, 3>, 3, 64);
-        }
-        break;
-      case 256: go(qk_norm_rope_fast_kernel<256, 2, 3>, 3, 64); break;
+      case 64: qk_norm_rope_warp_kernel<64, 2, 3><<<gw, kFastThreads, 0, stream>>>(p); break;
+      case 128: qk_norm_rope_warp_kernel<128, 2, 3><<<gw, kFastThreads, 0, stream>>>(p); break;
+      case 256: qk_norm_rope_warp_kernel<256, 2, 3><<<gw, kFastThreads, 0, stream>>>(p); break;
       default: return cudaErrorInvalidValue;
     }
   }

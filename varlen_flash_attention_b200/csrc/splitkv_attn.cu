@@ -60,7 +60,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sm_count = 0;
   int32_t* status = nullptr;
-  bool attn_attr_set[40] = {};  // per kernel instance: cudaFuncSetAttribute done
+  bool attn_attr_set[80] = {};  // per kernel instance: cudaFuncSetAttribute done
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -257,7 +257,7 @@ sk_status_t launch_attn(skattn::AttnParams& prm, int n_qtiles, int H, int nb, cu
                         DeviceInfo* dev) {
   const bool scatter = prm.out_chunk > 0;  // separate instance: the plain kernel's code is untouched
   const int variant = g_kernel_variant;
-  const int slot = (D == 64 ? 0 : 1) + (scatter ? 2 : 0) + 4 * variant;  // 0..23
+  const int slot = (D == 64 ? 0 : 1) + (scatter ? 2 : 0) + 4 * variant;  // 0..47
   sk_status_t st;
   if (variant == 2) {
     using L = skattn::SmemLayout<D>;
@@ -265,6 +265,26 @@ sk_status_t launch_attn(skattn::AttnParams& prm, int n_qtiles, int H, int nb, cu
     if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev)) != SK_OK) return st;
     dim3 grid(n_qtiles, H, nb);
     kernel<<<grid, skattn::kThreads, L::kAlloc, stream>>>(prm);
+  } else if (variant >= 9) {
+    // two threads per score row
+    using L = skattn::PSmemLayout<D, true>;
+    using P = skattn::AttnParams;
+    void (*kernel)(P) = nullptr;
+    switch (variant) {
+      case 10: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 2, P, false, true>; break;
+      case 11: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 3, P, false, true>; break;
+      default: kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, false, 0, P, false, true>
+                                : skattn::attn_fwd_persistent_kernel<D, false, false, 0, P, false, true>; break;
+    }
+    if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev, skattn::kSLaunchRegs)) != SK_OK)
+      return st;
+    prm.n_heads = H;
+    prm.n_pairs = n_qtiles;
+    const int64_t units = static_cast<int64_t>(nb) * H * n_qtiles;
+    if (units > INT32_MAX) return fail(SK_ERR_UNSUPPORTED, "too many work units (%lld)", (long long)units);
+    prm.n_units = static_cast<int32_t>(units);
+    const int grid = static_cast<int>(std::min<int64_t>(units, dev->sm_count));
+    kernel<<<grid, skattn::kSThreads, L::kAlloc, stream>>>(prm);
   } else {
     using L = skattn::PSmemLayout<D>;
     using P = skattn::AttnParams;
@@ -275,6 +295,9 @@ sk_status_t launch_attn(skattn::AttnParams& prm, int n_qtiles, int H, int nb, cu
       case 3: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 2, P>; break;
       case 4: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 3, P>; break;
       case 5: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 4, P>; break;
+      case 6: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 0, P, true>; break;
+      case 7: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 2, P, true>; break;
+      case 8: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 3, P, true>; break;
       default: kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, false, 0, P>
                                 : skattn::attn_fwd_persistent_kernel<D, false, false, 0, P>; break;
     }
@@ -434,7 +457,7 @@ template <int D>
 sk_status_t launch_varlen(skattn::VarlenParams& prm, cudaStream_t stream, DeviceInfo* dev) {
   using L = skattn::PSmemLayout<D>;
   const int variant = g_kernel_variant;
-  const int slot = 24 + (D == 64 ? 0 : 1) + 2 * (variant == 1);  // 24..27
+  const int slot = 64 + (D == 64 ? 0 : 1) + 2 * (variant == 1);  // 64..67
   auto kernel = variant == 1 ? skattn::attn_fwd_persistent_kernel<D, false, true, 0, skattn::VarlenParams>
                              : skattn::attn_fwd_persistent_kernel<D, false, false, 0, skattn::VarlenParams>;
   sk_status_t st;
@@ -788,7 +811,7 @@ sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, const vo
     prm.Hq = num_q_heads;
     prm.Hkv = num_kv_heads;
     prm.B = batch;
-    cudaError_t e = skqkn::launch(prm, head_dim, exact != 0, info->sm_count, static_cast<cudaStream_t>(stream));
+    cudaError_t e = skqkn::launch(prm, head_dim, exact != 0, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "qk_rmsnorm_rope launch");
     return SK_OK;
   } catch (...) {
@@ -833,16 +856,10 @@ sk_status_t sk_test_stall_mma(int32_t on) {
 
 int32_t sk_abi_version(void) { return kAbiVersion; }
 
-SK_API sk_status_t sk_debug_prologue_variant(int32_t v) {
-  if (v < 0 || v > 4) return fail(SK_ERR_INVALID_ARG, "variant must be in 0..4");
-  skqkn::fast_variant() = v;
-  return SK_OK;
-}
-
 // Development hook (not part of the header's interface): selects the
 // attention kernel variant for side-by-side timing.
 SK_API sk_status_t sk_debug_kernel_variant(int32_t v) {
-  if (v < 0 || v > 5) return fail(SK_ERR_INVALID_ARG, "variant must be in 0..5");
+  if (v < 0 || v > 11) return fail(SK_ERR_INVALID_ARG, "variant must be in 0..11");
   std::lock_guard<std::mutex> lk(g_mu);
   g_kernel_variant = v;
   return SK_OK;
