@@ -39,7 +39,8 @@ import workloads  # noqa: E402
 METRIC = "split-KV attention TFLOP/s and % of B200 dense-bf16 peak; max-abs err vs CPU oracle"
 DEFAULT_WORKLOAD = "long_gqa"
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = ["varlen_flash_attention_b200/csrc/attn_fwd_sm100.cuh",
+KERNEL_SOURCES = ["varlen_flash_attention_b200/csrc/attn_common.cuh",
+                  "varlen_flash_attention_b200/csrc/attn_fwd_persistent.cuh",
                   "varlen_flash_attention_b200/csrc/ptx.cuh",
                   "varlen_flash_attention_b200/csrc/splitkv_attn.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")

@@ -347,3 +347,38 @@ def test_fast_prologue_fused_view_leaves_v_untouched(sk):
     eps = float(np.float32(1e-5))
     _fast_check(_bits(got[:, :, :Hq]), qkv[:, :, :Hq].contiguous(), wq, tab, 96, False, eps)
     _fast_check(_bits(got[:, :, Hq:Hq + Hkv]), qkv[:, :, Hq:Hq + Hkv].contiguous(), wk, tab, 96, False, eps)
+
+
+@pytest.mark.parametrize("B,S,Hq,Hkv,D,rot,inter", [
+    (2, 333, 6, 2, 128, 96, False),      # fewer tokens than warps in the grid
+    (1, 4099, 32, 8, 128, 128, False),   # several tokens per warp, ragged tail
+    (1, 700, 16, 4, 64, 32, True),
+    (1, 300, 80, 8, 256, 128, False),    # many steps per token
+])
+def test_fast_prologue_contiguous_and_strided_heads_agree(sk, B, S, Hq, Hkv, D, rot, inter):
+    """The fp32 instance on contiguous heads and on heads spaced two rows
+    apart (a different address stream through the same copy ring): bit-
+    identical outputs, the rows in between untouched, both within the bound."""
+    gen = torch.Generator().manual_seed(B + S + Hq + D)
+    q = (torch.randn(B, S, Hq, D, generator=gen) * 1.5).to(torch.bfloat16)
+    k = torch.randn(B, S, Hkv, D, generator=gen).to(torch.bfloat16)
+    wq = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    wk = (1 + 0.1 * torch.randn(D, generator=gen)).to(torch.bfloat16)
+    tab = _table(S, rot)
+    qa, ka = q.cuda(), k.cuda()
+    qb_big = torch.zeros(B, S, 2 * Hq, D, dtype=torch.bfloat16, device="cuda")
+    kb_big = torch.zeros(B, S, 2 * Hkv, D, dtype=torch.bfloat16, device="cuda")
+    qb, kb = qb_big[:, :, ::2], kb_big[:, :, ::2]
+    qb.copy_(qa)
+    kb.copy_(ka)
+    args = (wq.cuda(), wk.cuda(), tab.cuda())
+    sk.qk_rmsnorm_rope(qa, ka, *args, rot_dim=rot, interleaved=inter, eps=1e-6)
+    sk.qk_rmsnorm_rope(qb, kb, *args, rot_dim=rot, interleaved=inter, eps=1e-6)
+    torch.cuda.synchronize()
+    assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+    # the rows between the strided heads are untouched
+    assert not qb_big[:, :, 1::2].any() and not kb_big[:, :, 1::2].any()
+    eps32 = float(np.float32(1e-6))
+    _fast_check(_bits(qa.cpu()), q, wq, tab, rot, inter, eps32)
+    _fast_check(_bits(ka.cpu()), k, wk, tab, rot, inter, eps32)

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = [os.path.join(HERE, "csrc", "splitkv_attn.cu")]
 DEPS = SOURCES + [
     os.path.join(HERE, "csrc", f)
-    for f in ("ptx.cuh", "attn_fwd_sm100.cuh", "qk_norm_rope.cuh", "shard_copy.cuh")
+    for f in ("ptx.cuh", "attn_common.cuh", "attn_fwd_persistent.cuh", "qk_norm_rope.cuh", "shard_copy.cuh")
 ] + [os.path.join(ROOT, "include", "splitkv_attn.h")]
 
 NVCC_FLAGS = [

@@ -17,7 +17,7 @@
 // Q load and first score MMAs overlap the previous unit's last PV MMAs and
 // epilogue.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads):
 //   warps 0-3  tile A, warps 4-7 tile B: thread t of a warpgroup owns query
 //              row t of its tile (TMEM lane t): loads its score row from
 //              TMEM, online softmax in fp32 (exp2, scale*log2 e folded in,
@@ -26,13 +26,14 @@
 //              of its own score row, and at the end of a unit reads O, divides
 //              by the row sum and stores the bf16 row.
 //   warp 8     TMA producer: Q tiles per unit, K and V tiles into rings.
-//   warp 9     TMEM allocator and tcgen05.mma issuer.  Per KV tile j the
+//   warp 9     TMEM allocator and tcgen05.mma issuer.
+//   warps 10-11 idle (they complete the third warpgroup, whose registers go
+//              to the softmax warpgroups).  Per KV tile j the
 //              order is PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): PV takes P from
 //              TMEM (A operand) and V from shared memory, so only K, V and Q
 //              are read from shared memory.  S_X(j+1) overwrites the columns
 //              PV_X(j) reads P from; it is issued behind PV_X(j) on the same
-//              in-order MMA pipe (kWaitPv = false) or once PV_X(j) has
-//              completed (kWaitPv = true).
+//              in-order MMA pipe, with no wait in between.
 // TMEM (512 columns): S_A/P_A [0,128), S_B/P_B [128,256), O_A [256,256+D),
 // O_B [384,384+D).
 // Every wait is bounded (globaltimer); on expiry the CTA raises the device
@@ -45,7 +46,7 @@
 #include <cstdint>
 #include <type_traits>
 
-#include "attn_fwd_sm100.cuh"
+#include "attn_common.cuh"
 #include "ptx.cuh"
 
 namespace skattn {
@@ -62,24 +63,14 @@ constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 224;
 constexpr int kOtherRegs = 56;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kPThreads * kLaunchRegs, "register split");
-// Two threads per row: 20 warps, 0-15 softmax (tile = warp / 8, column half =
-// (warp / 4) % 2), 16 TMA, 17 MMA, 18-19 idle; five warps per sub-partition
-// cap the launch at 96 registers: 4 * 128 * 104 + 128 * 64 = 640 * 96.
-constexpr int kSThreads = 640;
-constexpr int kSLaunchRegs = 96;
-constexpr int kSSoftmaxRegs = 104;
-constexpr int kSOtherRegs = 64;
-static_assert(4 * 128 * kSSoftmaxRegs + 128 * kSOtherRegs <= kSThreads * kSLaunchRegs, "register split");
 
-// kSplit: two threads per score row (the row maxima and sums are exchanged
-// through shared memory), which needs a smaller K ring to make room.
-template <int D, bool kSplit = false>
+template <int D>
 struct PSmemLayout {
   static_assert(D == 64 || D == 128, "head_dim");
   static constexpr uint32_t kSub = kBlockM * 128;  // one 64-column (128 B) swizzled sub-tile
   static constexpr uint32_t kQTile = kBlockM * D * 2;
   static constexpr uint32_t kKVTile = kBlockN * D * 2;
-  static constexpr int kKS = D == 128 ? (kSplit ? 2 : 3) : 4;  // K ring depth
+  static constexpr int kKS = D == 128 ? 3 : 4;  // K ring depth
   static constexpr int kVS = D == 128 ? 2 : 4;                 // V ring depth
   static constexpr uint32_t kQ = 0;                              // + tile * kQTile
   static constexpr uint32_t kK = kQ + kTilesPerCta * kQTile;     // + stage * kKVTile
@@ -95,13 +86,9 @@ struct PSmemLayout {
   static constexpr int bPLo = bSFull + 2;           // + tile: P_X(j) keys 0-63 in TMEM (128 arrivals)
   static constexpr int bPHi = bPLo + 2;             // + tile: P_X(j) keys 64-127 in TMEM (128 arrivals)
   static constexpr int bOFull = bPHi + 2;           // + tile: PV_X(last) of the unit finished
-  static constexpr int bPvDone = bOFull + 2;        // + tile: PV_X(j) finished (kWaitPv only)
-  static constexpr int bMmaDone = bPvDone + 2;
+  static constexpr int bMmaDone = bOFull + 2;
   static constexpr int kNumBars = bMmaDone + 1;
-  // kSplit: half-row maxima [tile][parity][half][row] and sums [tile][half][row]
-  static constexpr uint32_t kXm = kBar + kNumBars * 8;
-  static constexpr uint32_t kXl = kXm + (kSplit ? 2 * 2 * 2 * kBlockM * 4 : 0);
-  static constexpr uint32_t kMisc = kXl + (kSplit ? 2 * 2 * kBlockM * 4 : 0);
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;
   static constexpr uint32_t kEnd = kMisc + 16;
   static constexpr uint32_t kAlloc = (kEnd + 1024) > 120 * 1024 ? (kEnd + 1024) : 120 * 1024;
   static_assert(kAlloc <= 232448, "shared memory per CTA");
@@ -207,58 +194,10 @@ __device__ __forceinline__ uint16_t* unit_row_ptr(const VarlenParams& p, const P
   return p.out + static_cast<int64_t>(t.q_off + row) * p.out_ss + static_cast<int64_t>(t.hq) * p.out_sh;
 }
 
-// 2^x for a pair of values on the FMA pipe (the MUFU unit, which evaluates
-// ex2 for the other columns, runs at a quarter of the FMA rate).  Cody-Waite
-// split x = n + f, n = nearest integer (added to and removed from 1.5 * 2^23,
-// whose low mantissa bits then hold n), f in [-1/2, 1/2]; p(f) ~= 2^f is the
-// degree-3 polynomial of least maximum relative error on that interval
-// (Remez exchange, coefficients rounded to fp32, error 7.5e-5 -- below the
-// 2^-9 step of the bf16 P it feeds); 2^n is added to p's exponent field.
-// x is clamped at -126, so n >= -126 keeps the exponent field from wrapping
-// (results there are below 2^-125: zero for P in practice).
-__device__ __forceinline__ uint64_t exp2_fma_pipe(uint64_t x) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  float x0, x1;
-  skptx::f2_unpack(x, x0, x1);
-  x = skptx::f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t = skptx::add2(x, skptx::f2_pack(kMagic, kMagic));
-  const uint64_t f = skptx::sub2(x, skptx::sub2(t, skptx::f2_pack(kMagic, kMagic)));
-  uint64_t p = skptx::fma2(skptx::f2_pack(0x1.c3f76p-5f, 0x1.c3f76p-5f), f, skptx::f2_pack(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
-  p = skptx::fma2(p, f, skptx::f2_pack(0x1.62f31ap-1f, 0x1.62f31ap-1f));
-  p = skptx::fma2(p, f, skptx::f2_pack(0x1.fff692p-1f, 0x1.fff692p-1f));
-  float p0, p1, t0, t1;
-  skptx::f2_unpack(p, p0, p1);
-  skptx::f2_unpack(t, t0, t1);
-  return skptx::f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
-                        __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
-}
-
-// Which column pairs of each group of 8 take exp2 on the FMA pipe.
-template <int kPoly>
-__device__ __forceinline__ constexpr bool poly_pair(int i) {
-  return kPoly == 0 ? false
-       : kPoly == 2 ? (i % 8 == 2 || i % 8 == 6)
-       : kPoly == 3 ? (i % 8 == 1 || i % 8 == 4 || i % 8 == 6)
-       : (i % 2 == 1);
-}
-
-// Columns [32 * C0, 32 * C1) of one score row (already masked) -> P as bf16
-// pairs in TMEM columns tP + 16 * C0 .. tP + 16 * C1 - 1; returns the sum of
-// the fp32 exponentials p = 2^(s * sl2 - m).  Masked columns (partial tile)
-// are exact zeros.
-// Two non-negative finite fp32 values -> bf16 pair (lo in the low half),
-// rounded to nearest with ties away from zero: add half a bf16 ulp to each
-// bit pattern and keep the high halves.  Integer add and byte permute, so the
-// conversion stays off the MUFU pipe (the exponentials' bottleneck), where
-// the cvt.rn.bf16x2 instruction runs.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 // Columns [32 * C, 32 * C + 32) of one score row (already masked) -> 16 bf16
 // pairs of p = 2^(s * sl2 - m) in pk, their fp32 sum added to acc.  Masked
 // columns (partial tile) are exact zeros.
-template <int kPoly, bool kPartial, bool kIntPack, int C, int N>
+template <bool kPartial, int C, int N>
 __device__ __forceinline__ void exp_chunk(const float (&s)[N], uint64_t sl2_2, uint64_t negm_2, int nvalid,
                                           uint32_t (&pk)[16], uint64_t (&acc)[4]) {
   static_assert(32 * C + 32 <= N, "chunk inside the row");
@@ -266,20 +205,15 @@ __device__ __forceinline__ void exp_chunk(const float (&s)[N], uint64_t sl2_2, u
   for (int i = 0; i < 16; ++i) {
     const int c = C * 32 + 2 * i;
     const uint64_t x = skptx::fma2(skptx::f2_pack(s[c], s[c + 1]), sl2_2, negm_2);
-    float e0, e1;
-    if (poly_pair<kPoly>(i)) {
-      skptx::f2_unpack(exp2_fma_pipe(x), e0, e1);
-    } else {
-      float x0, x1;
-      skptx::f2_unpack(x, x0, x1);
-      e0 = skptx::ex2_approx(x0);
-      e1 = skptx::ex2_approx(x1);
-    }
+    float x0, x1;
+    skptx::f2_unpack(x, x0, x1);
+    float e0 = skptx::ex2_approx(x0);
+    float e1 = skptx::ex2_approx(x1);
     // exact zeros for masked columns (also when scale == 0: -inf * 0 is NaN)
     if (kPartial && c >= nvalid) e0 = 0.f;
     if (kPartial && c + 1 >= nvalid) e1 = 0.f;
     acc[i % 4] = skptx::add2(acc[i % 4], skptx::f2_pack(e0, e1));
-    pk[i] = kIntPack ? pack_bf16x2_int(e0, e1) : skptx::pack_bf16x2(e0, e1);
+    pk[i] = skptx::pack_bf16x2(e0, e1);
   }
 }
 
@@ -288,7 +222,7 @@ __device__ __forceinline__ void exp_chunk(const float (&s)[N], uint64_t sl2_2, u
 // returns the row sum of the fp32 exponentials.  The exponentials of keys
 // 64-95 are computed before the wait that releases keys 0-63, so that wait
 // finds the first stores already done.
-template <int kPoly, bool kPartial, bool kIntPack>
+template <bool kPartial>
 __device__ __forceinline__ float exp_row_release(const float (&s)[kBlockN], float sl2, float m, int nvalid,
                                                  uint32_t tP, uint32_t bar_lo, uint32_t bar_hi) {
   const uint64_t sl2_2 = skptx::f2_pack(sl2, sl2);
@@ -297,16 +231,16 @@ __device__ __forceinline__ float exp_row_release(const float (&s)[kBlockN], floa
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = 0;
   uint32_t pa[16], pb[16];
-  exp_chunk<kPoly, kPartial, kIntPack, 0>(s, sl2_2, negm_2, nvalid, pa, acc);
+  exp_chunk<kPartial, 0>(s, sl2_2, negm_2, nvalid, pa, acc);
   skptx::tmem_st16(tP, pa);
-  exp_chunk<kPoly, kPartial, kIntPack, 1>(s, sl2_2, negm_2, nvalid, pb, acc);
+  exp_chunk<kPartial, 1>(s, sl2_2, negm_2, nvalid, pb, acc);
   skptx::tmem_st16(tP + 16, pb);
-  exp_chunk<kPoly, kPartial, kIntPack, 2>(s, sl2_2, negm_2, nvalid, pa, acc);
+  exp_chunk<kPartial, 2>(s, sl2_2, negm_2, nvalid, pa, acc);
   skptx::tmem_wait_st();
   skptx::tc_fence_before();
   skptx::mbar_arrive(bar_lo);
   skptx::tmem_st16(tP + 32, pa);
-  exp_chunk<kPoly, kPartial, kIntPack, 3>(s, sl2_2, negm_2, nvalid, pb, acc);
+  exp_chunk<kPartial, 3>(s, sl2_2, negm_2, nvalid, pb, acc);
   skptx::tmem_st16(tP + 48, pb);
   skptx::tmem_wait_st();
   skptx::tc_fence_before();
@@ -334,7 +268,7 @@ __device__ __forceinline__ float half_max(const float (&s)[kBlockN]) {
 // (64-column sub-tiles kSub bytes apart).  Warp-collective.
 template <int D>
 __device__ __forceinline__ void issue_s_p(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
-  using L = PSmemLayout<D, false>;
+  using L = PSmemLayout<D>;
   constexpr uint32_t idS = skptx::idesc_bf16_f32(kBlockM, kBlockN, false);
   skptx::mma_ss_block<D / 16, (L::kSub >> 4)>(d_tmem, q_desc, k_desc, idS, 0u);
 }
@@ -369,9 +303,9 @@ __device__ __forceinline__ void zero_v_rows(uint32_t vbase, int r0, int r1, int 
 
 // The kernel's shared context: shared-memory base, TMEM base, the bounded
 // waiter and the barrier array (index -> shared address).
-template <int D, bool kSplit>
+template <int D>
 struct PCtx {
-  using L = PSmemLayout<D, kSplit>;
+  using L = PSmemLayout<D>;
   uint32_t sbase;
   uint32_t tmem;
   Waiter W;
@@ -380,9 +314,9 @@ struct PCtx {
 
 // ---------------------------------------------------------------- TMA producer
 // Q tiles per unit, K and V tiles into rings, in the order the MMAs need them.
-template <int D, bool kSplit, typename Params>
-__device__ __forceinline__ void tma_producer(const Params& p, const PCtx<D, kSplit>& cx, int lane) {
-  using L = PSmemLayout<D, kSplit>;
+template <int D, typename Params>
+__device__ __forceinline__ void tma_producer(const Params& p, const PCtx<D>& cx, int lane) {
+  using L = PSmemLayout<D>;
   constexpr bool kShared = std::is_same<Params, VarlenParams>::value;
   constexpr int KS = L::kKS;
   constexpr int VS = L::kVS;
@@ -456,9 +390,9 @@ __device__ __forceinline__ void tma_producer(const Params& p, const PCtx<D, kSpl
 // ---------------------------------------------------------------- MMA issuer
 // Per KV tile j: PV_A(j) (in two halves as P_A(j) is released), S_A(j+1),
 // PV_B(j), S_B(j+1).
-template <int D, bool kSplit, bool kWaitPv, typename Params>
-__device__ __forceinline__ void mma_issuer(const Params& p, const PCtx<D, kSplit>& cx, int lane) {
-  using L = PSmemLayout<D, kSplit>;
+template <int D, typename Params>
+__device__ __forceinline__ void mma_issuer(const Params& p, const PCtx<D>& cx, int lane) {
+  using L = PSmemLayout<D>;
   constexpr bool kShared = std::is_same<Params, VarlenParams>::value;
   constexpr int KS = L::kKS;
   constexpr int VS = L::kVS;
@@ -479,7 +413,6 @@ __device__ __forceinline__ void mma_issuer(const Params& p, const PCtx<D, kSplit
   int kc = 0, vc = 0;       // K / V ring positions consumed
   int un = 0;               // computed units so far (Q / O phases)
   int pc[2] = {0, 0};       // P tiles consumed per tile (PFull phases)
-  int pv[2] = {0, 0};       // PV MMAs committed to PvDone per tile
   auto wait_k = [&]() -> bool {
     return W.wait_warp(bar(L::bKFull + kc % KS), (kc / KS) & 1);
   };
@@ -488,13 +421,6 @@ __device__ __forceinline__ void mma_issuer(const Params& p, const PCtx<D, kSplit
     if (!t.compute) continue;
     const int n = t.n_tiles;
     if (!W.wait_warp(bar(L::bQFull + 0), un & 1) || !W.wait_warp(bar(L::bQFull + 1), un & 1) || !wait_k()) {
-      ok = false;
-      break;
-    }
-    // kWaitPv: S_X(0) overwrites the columns the previous unit's last PV_X
-    // read P from; wait for that PV (its OFull commit) first.
-    if (kWaitPv && un > 0 &&
-        (!W.wait_warp(bar(L::bOFull + 0), (un - 1) & 1) || !W.wait_warp(bar(L::bOFull + 1), (un - 1) & 1))) {
       ok = false;
       break;
     }
@@ -513,6 +439,7 @@ __device__ __forceinline__ void mma_issuer(const Params& p, const PCtx<D, kSplit
       const uint64_t dVs = dV + ((vs * L::kKVTile) >> 4);
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
+        const uint64_t dQx = dQ + ((x * L::kQTile) >> 4);
         // P arrives in two halves (keys 0-63, then 64-127): the first half
         // of PV runs while the softmax still exponentiates the second.
         if (!W.wait_warp(bar(L::bPLo + x), pc[x] & 1)) { ok = false; break; }
@@ -537,14 +464,9 @@ __device__ __forceinline__ void mma_issuer(const Params& p, const PCtx<D, kSplit
         }
         if (j == n - 1) skptx::mma_commit_elect(bar(L::bOFull + x));
         if (j + 1 < n) {
-          if (kWaitPv) {
-            skptx::mma_commit_elect(bar(L::bPvDone + x));
-            if (!W.wait_warp(bar(L::bPvDone + x), pv[x] & 1)) { ok = false; break; }
-            ++pv[x];
-          }
           if (x == 0 && !wait_k()) { ok = false; break; }
           skptx::tc_fence_after();
-          issue_s_p<D>(tS[x], dQ + ((x * L::kQTile) >> 4), dK + (((kc % KS) * L::kKVTile) >> 4));
+          issue_s_p<D>(tS[x], dQx, dK + (((kc % KS) * L::kKVTile) >> 4));
           skptx::mma_commit_elect(bar(L::bSFull + x));
           if (j + 1 == n - 1) skptx::mma_commit_elect(bar(L::bQEmpty + x));
           if (x == 1) {
@@ -565,9 +487,9 @@ __device__ __forceinline__ void mma_issuer(const Params& p, const PCtx<D, kSplit
 // ---------------------------------------------------------------- softmax, one thread per row
 // Warps 0-3 tile A, 4-7 tile B: thread t of a warpgroup owns query row t of
 // its tile (TMEM lane t) and all 128 columns of its score row.
-template <int D, bool kScatter, int kPoly, bool kIntPack, typename Params>
-__device__ __forceinline__ void softmax_rows(const Params& p, const PCtx<D, false>& cx, int warp) {
-  using L = PSmemLayout<D, false>;
+template <int D, bool kScatter, typename Params>
+__device__ __forceinline__ void softmax_rows(const Params& p, const PCtx<D>& cx, int warp) {
+  using L = PSmemLayout<D>;
   const uint32_t tmem = cx.tmem;
   const Waiter& W = cx.W;
   auto bar = [&](int i) { return cx.bar(i); };
@@ -642,9 +564,8 @@ __device__ __forceinline__ void softmax_rows(const Params& p, const PCtx<D, fals
           skptx::tmem_st32(tO + c * 32, o);
         }
       }
-      const float sum =
-          partial ? exp_row_release<kPoly, true, kIntPack>(s, sl2, m_run, nvalid, tS_, bar(L::bPLo + x), bar(L::bPHi + x))
-                  : exp_row_release<kPoly, false, kIntPack>(s, sl2, m_run, nvalid, tS_, bar(L::bPLo + x), bar(L::bPHi + x));
+      const float sum = partial ? exp_row_release<true>(s, sl2, m_run, nvalid, tS_, bar(L::bPLo + x), bar(L::bPHi + x))
+                                : exp_row_release<false>(s, sl2, m_run, nvalid, tS_, bar(L::bPLo + x), bar(L::bPHi + x));
       l_run = l_run * alpha + sum;
     }
     if (!ok) break;
@@ -685,234 +606,16 @@ __device__ __forceinline__ void softmax_rows(const Params& p, const PCtx<D, fals
   }
 }
 
-// Columns [32 C, 32 C + 32) of a 64-column half row -> P in TMEM columns
-// tP + 16 C .. tP + 16 C + 15, stored 8 columns at a time (fewer live
-// registers), their fp32 sum added to the two accumulators.
-template <int kPoly, bool kPartial, int C>
-__device__ __forceinline__ void exp_chunk_half(const float (&s)[64], uint64_t sl2_2, uint64_t negm_2, int nvalid,
-                                               uint32_t tP, uint64_t (&acc)[2]) {
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    uint32_t pk[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = C * 32 + q * 16 + 2 * i;
-      const uint64_t x = skptx::fma2(skptx::f2_pack(s[c], s[c + 1]), sl2_2, negm_2);
-      float e0, e1;
-      if (poly_pair<kPoly>(q * 8 + i)) {
-        skptx::f2_unpack(exp2_fma_pipe(x), e0, e1);
-      } else {
-        float x0, x1;
-        skptx::f2_unpack(x, x0, x1);
-        e0 = skptx::ex2_approx(x0);
-        e1 = skptx::ex2_approx(x1);
-      }
-      if (kPartial && c >= nvalid) e0 = 0.f;
-      if (kPartial && c + 1 >= nvalid) e1 = 0.f;
-      acc[i % 2] = skptx::add2(acc[i % 2], skptx::f2_pack(e0, e1));
-      pk[i] = skptx::pack_bf16x2(e0, e1);
-    }
-    skptx::tmem_st8(tP + C * 16 + q * 8, pk);
-  }
-}
-
-// ---------------------------------------------------------------- softmax, two threads per row
-// Warps 0-15: tile x = warp / 8, column half h = (warp / 4) % 2; thread t of
-// a warpgroup owns columns [64h, 64h + 64) of query row t of its tile (both
-// halves of a row sit in the same TMEM lane, read by warps of the same lane
-// quarter).  Per tile the halves exchange their row maxima through shared
-// memory at one named barrier (which also ANDs their wait results, so the two
-// halves always leave the loop together); each half writes its 32 columns of
-// P and releases them on its own barrier (PLo / PHi), rescales and finally
-// stores its 64 (D / 2) output columns.
-template <int D, bool kScatter, int kPoly, bool kIntPack, typename Params>
-__device__ __forceinline__ void softmax_halves(const Params& p, const PCtx<D, true>& cx, int warp) {
-  using L = PSmemLayout<D, true>;
-  constexpr int DH = D / 2;  // output columns per half
-  const uint32_t tmem = cx.tmem;
-  const Waiter& W = cx.W;
-  auto bar = [&](int i) { return cx.bar(i); };
-  const int n_units = p.n_units;
-  const int x = warp / 8;
-  const int h = (warp / 4) % 2;
-  const int r = threadIdx.x % 128;
-  const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
-  const uint32_t tS_ = tmem + lane_base + static_cast<uint32_t>(x) * 128 + h * 64;  // this half's scores
-  const uint32_t tP_ = tmem + lane_base + static_cast<uint32_t>(x) * 128 + h * 32;  // this half's P (bf16 pairs)
-  const uint32_t tO = tmem + lane_base + 256 + static_cast<uint32_t>(x) * 128 + h * DH;
-  const uint32_t xm_mine = cx.sbase + L::kXm + static_cast<uint32_t>(((x * 2) * 2 + h) * kBlockM + r) * 4;
-  const uint32_t xm_other = cx.sbase + L::kXm + static_cast<uint32_t>(((x * 2) * 2 + (1 - h)) * kBlockM + r) * 4;
-  constexpr uint32_t kXmParity = 2 * kBlockM * 4;  // bytes between the parity slots of a tile
-  const uint32_t xl_mine = cx.sbase + L::kXl + static_cast<uint32_t>((x * 2 + h) * kBlockM + r) * 4;
-  const uint32_t xl_other = cx.sbase + L::kXl + static_cast<uint32_t>((x * 2 + (1 - h)) * kBlockM + r) * 4;
-  const uint32_t bar_id = 1 + x;  // named barrier of the tile's 8 warps
-  const float sl2 = p.scale_log2;
-  int sc = 0;  // score tiles consumed (SFull phases, exchange parity)
-  int un = 0;  // computed units so far (OFull phases)
-  bool ok = true;
-  for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
-    const PUnit t = decode_unit(p, u);
-    const int row = t.row0 + x * kBlockM + r;
-    if (!t.compute) {
-      if (row < t.sq) {
-        uint4* dst = reinterpret_cast<uint4*>(unit_row_ptr<kScatter>(p, t, row) + h * DH);
-#pragma unroll
-        for (int v = 0; v < DH / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
-      }
-      continue;
-    }
-    float m_run = 0.f;  // running (possibly stale) max of scale*log2(e)*s, shared by both halves
-    float l_run = 0.f;  // this half's running sum of exponentials
-    for (int j = 0; j < t.n_tiles; ++j) {
-      const uint32_t par = static_cast<uint32_t>(sc & 1);
-      bool waited = W.wait_warp(bar(L::bSFull + x), par);
-      ++sc;
-      skptx::tc_fence_after();
-      const int nvalid = tile_valid(j, t.tP, t.nkp, t.nks) - h * 64;  // valid columns of this half
-      const bool partial = nvalid < 64;
-      // (after a failed wait the values are garbage, but the loop is left
-      // at the barrier below before they are used)
-      float s[64];
-      {
-        uint32_t uu[2][32];
-        skptx::tmem_ld32(tS_, uu[0]);
-        skptx::tmem_ld32(tS_ + 32, uu[1]);
-        skptx::tmem_wait_ld();
-        skptx::reg_fence(uu[0]);
-        skptx::reg_fence(uu[1]);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(uu[c / 32][c % 32]);
-      }
-      if (partial) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= nvalid) s[c] = -INFINITY;
-      }
-      float mx[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        mx[k] = fmaxf(s[k], s[k + 4]);
-#pragma unroll
-        for (int c = 8 + k; c < 64; c += 8) mx[k] = skptx::fmax3(mx[k], s[c], s[c + 4]);
-      }
-      skptx::st_shared_f32(xm_mine + par * kXmParity, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
-      // The barrier also orders this half's TMEM loads before the other
-      // half's P stores: half 1 writes P over score columns 32-63, which
-      // half 0 reads.
-      skptx::tc_fence_before();
-      ok = skptx::bar_and(bar_id, 256, waited);
-      skptx::tc_fence_after();
-      if (!ok) break;
-      const float m_tile =
-          fmaxf(skptx::ld_shared_f32(xm_mine + par * kXmParity), skptx::ld_shared_f32(xm_other + par * kXmParity)) * sl2;
-      float alpha = 1.f;
-      bool raise = false;
-      if (j == 0) {
-        m_run = m_tile;
-      } else if (m_tile > m_run + kRescaleLog2) {
-        alpha = skptx::ex2_approx(m_run - m_tile);
-        m_run = m_tile;
-        raise = true;
-      }
-      // O_X holds the sum over tiles < j (PV_X(j-1) finished before S_X(j)
-      // was complete); each half rescales its own output columns (rare: only
-      // when the row maximum grows by more than 2^kRescaleLog2; both halves
-      // of a row take the same decision), 8 columns at a time to keep few
-      // registers live beside the scores.  Every PV step writes all output
-      // columns, so PLo counts both halves: half 1 arrives there as soon as
-      // its columns are rescaled (or at once), half 0 once its P is stored.
-      if (__any_sync(0xffffffffu, raise)) {
-#pragma unroll 1
-        for (int c = 0; c < DH / 8; ++c) {
-          uint32_t o[8];
-          skptx::tmem_ld8(tO + c * 8, o);
-          skptx::tmem_wait_ld();
-          skptx::reg_fence(o);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          skptx::tmem_st8(tO + c * 8, o);
-        }
-      }
-      if (h == 1) {
-        skptx::tmem_wait_st();
-        skptx::tc_fence_before();
-        skptx::mbar_arrive(bar(L::bPLo + x));
-      }
-      const uint64_t sl2_2 = skptx::f2_pack(sl2, sl2);
-      const uint64_t negm_2 = skptx::f2_pack(-m_run, -m_run);
-      uint64_t acc[2] = {0, 0};
-      if (partial) {
-        exp_chunk_half<kPoly, true, 0>(s, sl2_2, negm_2, nvalid, tP_, acc);
-        exp_chunk_half<kPoly, true, 1>(s, sl2_2, negm_2, nvalid, tP_, acc);
-      } else {
-        exp_chunk_half<kPoly, false, 0>(s, sl2_2, negm_2, nvalid, tP_, acc);
-        exp_chunk_half<kPoly, false, 1>(s, sl2_2, negm_2, nvalid, tP_, acc);
-      }
-      skptx::tmem_wait_st();
-      skptx::tc_fence_before();
-      if (h == 0) skptx::mbar_arrive(bar(L::bPLo + x));
-      skptx::mbar_arrive(bar(L::bPHi + x));
-      const uint64_t a = skptx::add2(acc[0], acc[1]);
-      float a0, a1;
-      skptx::f2_unpack(a, a0, a1);
-      l_run = l_run * alpha + (a0 + a1);
-    }
-    if (!ok) break;
-    // ---------------------------------------------------------- epilogue
-    const PUnit te = decode_unit(p, u);  // recomputed: fewer registers live through the tile loop
-    const bool waited = W.wait_warp(bar(L::bOFull + x), un & 1);
-    ++un;
-    skptx::st_shared_f32(xl_mine, l_run);
-    skptx::tc_fence_before();
-    ok = skptx::bar_and(bar_id, 256, waited);
-    skptx::tc_fence_after();
-    if (!ok) break;
-    const float l_row = skptx::ld_shared_f32(xl_mine) + skptx::ld_shared_f32(xl_other);
-    const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
-    const int erow = te.row0 + x * kBlockM + r;
-    uint16_t* orow = unit_row_ptr<kScatter>(p, te, erow < te.sq ? erow : 0) + h * DH;
-#pragma unroll
-    for (int c = 0; c < DH / 32; ++c) {
-      uint32_t o[32];
-      skptx::tmem_ld32(tO + c * 32, o);
-      skptx::tmem_wait_ld();
-      skptx::reg_fence(o);
-      if (erow < te.sq) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-        if (erow < te.qv) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = skptx::pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-            w.y = skptx::pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-            w.z = skptx::pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-            w.w = skptx::pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-            dst[v] = w;
-          }
-        } else {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(0, 0, 0, 0);
-        }
-      }
-    }
-    skptx::tc_fence_before();
-  }
-}
-
 // ---------------------------------------------------------------- the kernel
 // Params: AttnParams (batch rows, split K/V) or VarlenParams (packed segments).
-// kPoly: column pairs of every 8 whose exponentials run on the FMA pipe;
-// kIntPack: P rounded to bf16 with integer operations (off the MUFU pipe);
-// kSplit: two threads per score row (20 warps) instead of one (12 warps).
-template <int D, bool kScatter, bool kWaitPv, int kPoly, typename Params, bool kIntPack = false, bool kSplit = false>
-__global__ void __launch_bounds__(kSplit ? kSThreads : kPThreads, 1)
-    attn_fwd_persistent_kernel(const __grid_constant__ Params p) {
-  using L = PSmemLayout<D, kSplit>;
+template <int D, bool kScatter, typename Params>
+__global__ void __launch_bounds__(kPThreads, 1) attn_fwd_persistent_kernel(const __grid_constant__ Params p) {
+  using L = PSmemLayout<D>;
   constexpr int KS = L::kKS;
   constexpr int VS = L::kVS;
-  constexpr int kTma = kSplit ? 16 : 8;
-  constexpr int kMma = kSplit ? 17 : 9;
-  constexpr int kSoftWarps = kSplit ? 16 : 8;
+  constexpr int kTma = 8;
+  constexpr int kMma = 9;
+  constexpr int kSoftWarps = 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -928,10 +631,9 @@ __global__ void __launch_bounds__(kSplit ? kSThreads : kPThreads, 1)
       skptx::mbar_init(bar(L::bQFull + x), 1);
       skptx::mbar_init(bar(L::bQEmpty + x), 1);
       skptx::mbar_init(bar(L::bSFull + x), 1);
-      skptx::mbar_init(bar(L::bPLo + x), kSplit ? 2 * kBlockM : kBlockM);
-      skptx::mbar_init(bar(L::bPHi + x), kSplit ? 2 * kBlockM : kBlockM);
+      skptx::mbar_init(bar(L::bPLo + x), kBlockM);
+      skptx::mbar_init(bar(L::bPHi + x), kBlockM);
       skptx::mbar_init(bar(L::bOFull + x), 1);
-      skptx::mbar_init(bar(L::bPvDone + x), 1);
     }
     for (int s = 0; s < KS; ++s) {
       skptx::mbar_init(bar(L::bKFull + s), 1);
@@ -952,17 +654,16 @@ __global__ void __launch_bounds__(kSplit ? kSThreads : kPThreads, 1)
   skptx::tc_fence_before();
   __syncthreads();
   skptx::tc_fence_after();
-  const PCtx<D, kSplit> cx{sbase, *tmem_slot, Waiter{abort_flag, p.status, p.wait_limit_ns}};
+  const PCtx<D> cx{sbase, *tmem_slot, Waiter{abort_flag, p.status, p.wait_limit_ns}};
   // Each role sets its register budget at the top of its own branch (the
   // compiler allocates every branch within the budget it sets).
   if (warp >= kSoftWarps) {
-    skptx::setmaxnreg_dec<kSplit ? kSOtherRegs : kOtherRegs>();
-    if (warp == kTma) tma_producer<D, kSplit>(p, cx, lane);
-    else if (warp == kMma) mma_issuer<D, kSplit, kWaitPv>(p, cx, lane);
+    skptx::setmaxnreg_dec<kOtherRegs>();
+    if (warp == kTma) tma_producer<D>(p, cx, lane);
+    else if (warp == kMma) mma_issuer<D>(p, cx, lane);
   } else {
-    skptx::setmaxnreg_inc<kSplit ? kSSoftmaxRegs : kSoftmaxRegs>();
-    if constexpr (kSplit) softmax_halves<D, kScatter, kPoly, kIntPack>(p, cx, warp);
-    else softmax_rows<D, kScatter, kPoly, kIntPack>(p, cx, warp);
+    skptx::setmaxnreg_inc<kSoftmaxRegs>();
+    softmax_rows<D, kScatter>(p, cx, warp);
   }
 
   skptx::tc_fence_before();

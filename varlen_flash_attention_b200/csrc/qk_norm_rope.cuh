@@ -358,7 +358,8 @@ constexpr int kFastThreads = 256;
 // fp32 instance, one token per warp: 32 / (D/8) rows per load instruction,
 // so a warp streams through its token's heads in contiguous runs (BATCH
 // loads of (32 / (D/8)) consecutive heads per iteration, the next batch in
-// flight).
+// flight).  One block per kFastThreads / 32 tokens, MINB blocks per SM: the
+// bytes in flight per SM are set by the warps resident and BATCH.
 template <int D, int BATCH, int MINB>
 __global__ void __launch_bounds__(kFastThreads, MINB) qk_norm_rope_warp_kernel(const NormRopeParams p) {
   constexpr int TPR = D / 8;            // lanes per row
@@ -373,17 +374,25 @@ __global__ void __launch_bounds__(kFastThreads, MINB) qk_norm_rope_warp_kernel(c
   const int sub = lane % TPR;
   const int g = lane / TPR;             // row within a warp-wide load
   const int d0 = sub * 8;
-  const int64_t tok = static_cast<int64_t>(blockIdx.x) * (kFastThreads / 32) + threadIdx.x / 32;
-  const bool valid = tok < static_cast<int64_t>(p.B) * p.S;
-  const int s = valid ? static_cast<int>(tok % p.S) : 0;
-  const int b = valid ? static_cast<int>(tok / p.S) : 0;
   const int rot = p.rot_dim;
   const bool rotates = d0 < rot;
+  int src = lane;
+  if (!p.interleaved && rot > 0) {
+    const int half = rot / 2, hs = half / 8;
+    if (d0 < half) src = lane + hs;
+    else if (d0 < rot) src = lane - hs;
+  }
+  const int H = p.Hq + p.Hkv;
+  const float inv_d = 1.0f / static_cast<float>(D);
+  const int64_t n_tok = static_cast<int64_t>(p.B) * p.S;
+  const int64_t tok = static_cast<int64_t>(blockIdx.x) * (kFastThreads / 32) + threadIdx.x / 32;
+  if (tok >= n_tok) return;  // whole warps: every shuffle below has all 32 lanes
+  const int s = static_cast<int>(tok % p.S);
+  const int b = static_cast<int>(tok / p.S);
   float c[8], sg[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) { c[i] = 1.0f; sg[i] = 0.0f; }
-  int src = lane;
-  if (rotates && valid) {
+  if (rotates) {
     const float* crow = p.table + static_cast<int64_t>(s) * rot;
     if (p.interleaved) {
       const float4 c4 = *reinterpret_cast<const float4*>(crow + d0 / 2);
@@ -413,29 +422,22 @@ __global__ void __launch_bounds__(kFastThreads, MINB) qk_norm_rope_warp_kernel(c
       }
     }
   }
-  if (!p.interleaved && rot > 0) {
-    const int half = rot / 2, hs = half / 8;
-    if (d0 < half) src = lane + hs;
-    else if (d0 < rot) src = lane - hs;
-  }
-  const int H = p.Hq + p.Hkv;
   uint16_t* qrow = p.q + b * p.q_sb + s * p.q_ss + d0;
   uint16_t* krow = p.k + b * p.k_sb + s * p.k_ss + d0 - static_cast<int64_t>(p.Hq) * p.k_sh;
   auto row_ptr = [&](int h) { return h < p.Hq ? qrow + h * p.q_sh : krow + h * p.k_sh; };
-  const float inv_d = 1.0f / static_cast<float>(D);
 
   uint4 xv[BATCH];
 #pragma unroll
   for (int j = 0; j < BATCH; ++j) {
     const int h = g + RPW * j;
-    xv[j] = (valid && h < H) ? *reinterpret_cast<const uint4*>(row_ptr(h)) : make_uint4(0, 0, 0, 0);
+    xv[j] = h < H ? *reinterpret_cast<const uint4*>(row_ptr(h)) : make_uint4(0, 0, 0, 0);
   }
   for (int h0 = 0; h0 < H; h0 += STEP) {
     uint4 xn[BATCH];
 #pragma unroll
     for (int j = 0; j < BATCH; ++j) {
       const int h = h0 + STEP + g + RPW * j;
-      xn[j] = (valid && h < H) ? *reinterpret_cast<const uint4*>(row_ptr(h)) : make_uint4(0, 0, 0, 0);
+      xn[j] = h < H ? *reinterpret_cast<const uint4*>(row_ptr(h)) : make_uint4(0, 0, 0, 0);
     }
     float ss[BATCH];
 #pragma unroll
@@ -483,12 +485,13 @@ __global__ void __launch_bounds__(kFastThreads, MINB) qk_norm_rope_warp_kernel(c
         const float zc = fmaf(bf16_hi(pb[i]), sg[2 * i + 1], bf16_hi(yb[i]) * c[2 * i + 1]);
         zb[i] = rotates ? pack_bf16x2_rn(za, zc) : yb[i];
       }
-      if (valid && h < H) *reinterpret_cast<uint4*>(row_ptr(h)) = make_uint4(zb[0], zb[1], zb[2], zb[3]);
+      if (h < H) *reinterpret_cast<uint4*>(row_ptr(h)) = make_uint4(zb[0], zb[1], zb[2], zb[3]);
     }
 #pragma unroll
     for (int j = 0; j < BATCH; ++j) xv[j] = xn[j];
   }
 }
+
 
 inline cudaError_t launch(const NormRopeParams& p, int D, bool exact, cudaStream_t stream) {
   const int64_t tokens = static_cast<int64_t>(p.B) * p.S;
@@ -504,17 +507,17 @@ inline cudaError_t launch(const NormRopeParams& p, int D, bool exact, cudaStream
       case 256: qk_norm_rope_kernel<256><<<g, kNormRopeThreads, 0, stream>>>(p); break;
       default: return cudaErrorInvalidValue;
     }
-  } else {
-    // one token per warp, kFastThreads / 32 tokens per block
-    const int64_t wblocks = (tokens + kFastThreads / 32 - 1) / (kFastThreads / 32);
-    if (wblocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    const unsigned gw = static_cast<unsigned>(wblocks);
-    switch (D) {
-      case 64: qk_norm_rope_warp_kernel<64, 2, 3><<<gw, kFastThreads, 0, stream>>>(p); break;
-      case 128: qk_norm_rope_warp_kernel<128, 2, 3><<<gw, kFastThreads, 0, stream>>>(p); break;
-      case 256: qk_norm_rope_warp_kernel<256, 2, 3><<<gw, kFastThreads, 0, stream>>>(p); break;
-      default: return cudaErrorInvalidValue;
-    }
+    return cudaGetLastError();
+  }
+  // one token per warp, kFastThreads / 32 tokens per block, 4 blocks per SM
+  const int64_t wblocks = (tokens + kFastThreads / 32 - 1) / (kFastThreads / 32);
+  if (wblocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  const unsigned gw = static_cast<unsigned>(wblocks);
+  switch (D) {
+    case 64: qk_norm_rope_warp_kernel<64, 2, 4><<<gw, kFastThreads, 0, stream>>>(p); break;
+    case 128: qk_norm_rope_warp_kernel<128, 2, 4><<<gw, kFastThreads, 0, stream>>>(p); break;
+    case 256: qk_norm_rope_warp_kernel<256, 2, 4><<<gw, kFastThreads, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }

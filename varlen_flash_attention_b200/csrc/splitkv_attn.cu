@@ -18,7 +18,7 @@
 #include <cstddef>
 
 #include "../../include/splitkv_attn.h"
-#include "attn_fwd_sm100.cuh"
+#include "attn_common.cuh"
 #include "attn_fwd_persistent.cuh"
 #include "qk_norm_rope.cuh"
 #include "shard_copy.cuh"
@@ -50,9 +50,6 @@ __device__ int32_t g_device_status = 0;
 
 uint64_t g_wait_limit_ns = 2000ull * 1000ull * 1000ull;
 int32_t g_test_stall = 0;
-// Attention kernel: 0 = persistent, P in TMEM, S(j+1) queued behind PV(j);
-// 1 = the same waiting for PV(j) to finish; 2 = one CTA per 256-row block.
-int32_t g_kernel_variant = 0;
 std::mutex g_mu;
 
 struct DeviceInfo {
@@ -60,7 +57,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int sm_count = 0;
   int32_t* status = nullptr;
-  bool attn_attr_set[80] = {};  // per kernel instance: cudaFuncSetAttribute done
+  bool attn_attr_set[8] = {};  // per kernel instance: cudaFuncSetAttribute done
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -255,62 +252,21 @@ sk_status_t set_smem(const void* kernel, int slot, uint32_t bytes, DeviceInfo* d
 template <int D>
 sk_status_t launch_attn(skattn::AttnParams& prm, int n_qtiles, int H, int nb, cudaStream_t stream,
                         DeviceInfo* dev) {
+  using L = skattn::PSmemLayout<D>;
+  using P = skattn::AttnParams;
   const bool scatter = prm.out_chunk > 0;  // separate instance: the plain kernel's code is untouched
-  const int variant = g_kernel_variant;
-  const int slot = (D == 64 ? 0 : 1) + (scatter ? 2 : 0) + 4 * variant;  // 0..47
+  const int slot = (D == 64 ? 0 : 1) + (scatter ? 2 : 0);
+  auto kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, P> : skattn::attn_fwd_persistent_kernel<D, false, P>;
   sk_status_t st;
-  if (variant == 2) {
-    using L = skattn::SmemLayout<D>;
-    auto kernel = scatter ? skattn::attn_fwd_kernel<D, true> : skattn::attn_fwd_kernel<D, false>;
-    if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev)) != SK_OK) return st;
-    dim3 grid(n_qtiles, H, nb);
-    kernel<<<grid, skattn::kThreads, L::kAlloc, stream>>>(prm);
-  } else if (variant >= 9) {
-    // two threads per score row
-    using L = skattn::PSmemLayout<D, true>;
-    using P = skattn::AttnParams;
-    void (*kernel)(P) = nullptr;
-    switch (variant) {
-      case 10: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 2, P, false, true>; break;
-      case 11: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 3, P, false, true>; break;
-      default: kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, false, 0, P, false, true>
-                                : skattn::attn_fwd_persistent_kernel<D, false, false, 0, P, false, true>; break;
-    }
-    if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev, skattn::kSLaunchRegs)) != SK_OK)
-      return st;
-    prm.n_heads = H;
-    prm.n_pairs = n_qtiles;
-    const int64_t units = static_cast<int64_t>(nb) * H * n_qtiles;
-    if (units > INT32_MAX) return fail(SK_ERR_UNSUPPORTED, "too many work units (%lld)", (long long)units);
-    prm.n_units = static_cast<int32_t>(units);
-    const int grid = static_cast<int>(std::min<int64_t>(units, dev->sm_count));
-    kernel<<<grid, skattn::kSThreads, L::kAlloc, stream>>>(prm);
-  } else {
-    using L = skattn::PSmemLayout<D>;
-    using P = skattn::AttnParams;
-    void (*kernel)(P) = nullptr;
-    switch (variant) {
-      case 1: kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, true, 0, P>
-                               : skattn::attn_fwd_persistent_kernel<D, false, true, 0, P>; break;
-      case 3: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 2, P>; break;
-      case 4: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 3, P>; break;
-      case 5: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 4, P>; break;
-      case 6: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 0, P, true>; break;
-      case 7: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 2, P, true>; break;
-      case 8: kernel = skattn::attn_fwd_persistent_kernel<D, false, false, 3, P, true>; break;
-      default: kernel = scatter ? skattn::attn_fwd_persistent_kernel<D, true, false, 0, P>
-                                : skattn::attn_fwd_persistent_kernel<D, false, false, 0, P>; break;
-    }
-    if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev, skattn::kLaunchRegs)) != SK_OK)
-      return st;
-    prm.n_heads = H;
-    prm.n_pairs = n_qtiles;
-    const int64_t units = static_cast<int64_t>(nb) * H * n_qtiles;
-    if (units > INT32_MAX) return fail(SK_ERR_UNSUPPORTED, "too many work units (%lld)", (long long)units);
-    prm.n_units = static_cast<int32_t>(units);
-    const int grid = static_cast<int>(std::min<int64_t>(units, dev->sm_count));
-    kernel<<<grid, skattn::kPThreads, L::kAlloc, stream>>>(prm);
-  }
+  if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev, skattn::kLaunchRegs)) != SK_OK)
+    return st;
+  prm.n_heads = H;
+  prm.n_pairs = n_qtiles;
+  const int64_t units = static_cast<int64_t>(nb) * H * n_qtiles;
+  if (units > INT32_MAX) return fail(SK_ERR_UNSUPPORTED, "too many work units (%lld)", (long long)units);
+  prm.n_units = static_cast<int32_t>(units);
+  const int grid = static_cast<int>(std::min<int64_t>(units, dev->sm_count));
+  kernel<<<grid, skattn::kPThreads, L::kAlloc, stream>>>(prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
   return SK_OK;
@@ -456,10 +412,8 @@ sk_status_t attn_impl(const sk_tensor_t* q, const sk_tensor_t* kp, const sk_tens
 template <int D>
 sk_status_t launch_varlen(skattn::VarlenParams& prm, cudaStream_t stream, DeviceInfo* dev) {
   using L = skattn::PSmemLayout<D>;
-  const int variant = g_kernel_variant;
-  const int slot = 64 + (D == 64 ? 0 : 1) + 2 * (variant == 1);  // 64..67
-  auto kernel = variant == 1 ? skattn::attn_fwd_persistent_kernel<D, false, true, 0, skattn::VarlenParams>
-                             : skattn::attn_fwd_persistent_kernel<D, false, false, 0, skattn::VarlenParams>;
+  const int slot = 4 + (D == 64 ? 0 : 1);
+  auto kernel = skattn::attn_fwd_persistent_kernel<D, false, skattn::VarlenParams>;
   sk_status_t st;
   if ((st = set_smem<D>(reinterpret_cast<const void*>(kernel), slot, L::kAlloc, dev, skattn::kLaunchRegs)) != SK_OK)
     return st;
@@ -585,50 +539,7 @@ sk_status_t varlen_impl(const sk_tensor_t* q, const sk_tensor_t* k, const sk_ten
   DeviceInfo* info = nullptr;
   if ((st = device_setup(&dev, &info)) != SK_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-  if (g_kernel_variant != 2)
-    return varlen_persistent(q, k, v, cu_q, cu_k, used_q, used_k, nseg, Hq, Hkv, scale, out, D, stream, info);
-  auto rptr = [](const sk_tensor_t* t, int64_t row) {
-    return static_cast<const void*>(static_cast<const uint16_t*>(t->ptr) + row * t->stride_s);
-  };
-  for (int s0 = 0; s0 < nseg; s0 += skattn::kMaxBatch) {
-    const int nb = std::min(skattn::kMaxBatch, nseg - s0);
-    skattn::AttnParams prm;
-    std::memset(&prm, 0, sizeof prm);
-    int32_t chunk_sq = 0;
-    for (int i = 0; i < nb; ++i) {
-      const int g = s0 + i;
-      const int32_t lq = cu_q[g + 1] - cu_q[g];
-      const int32_t lk = cu_k[g + 1] - cu_k[g];
-      const int32_t nk = used_k ? used_k[g] : lk;
-      const int32_t qv = used_q ? used_q[g] : lq;
-      prm.q_valid[i] = qv;
-      prm.n_prefix[i] = 0;
-      prm.n_suffix[i] = nk;
-      prm.sq[i] = lq;
-      prm.out_off[i] = static_cast<int64_t>(cu_q[g]) * out->stride_s;
-      chunk_sq = std::max(chunk_sq, lq);
-      if (qv > 0 && nk > 0)
-        if ((st = encode_map(&prm.tm_q[i], rptr(q, cu_q[g]), q->stride_s, q->stride_h, Hq, qv, D)) != SK_OK) return st;
-      if (nk > 0) {
-        if ((st = encode_map(&prm.tm_ks[i], rptr(k, cu_k[g]), k->stride_s, k->stride_h, Hkv, nk, D)) != SK_OK) return st;
-        if ((st = encode_map(&prm.tm_vs[i], rptr(v, cu_k[g]), v->stride_s, v->stride_h, Hkv, nk, D)) != SK_OK) return st;
-      }
-    }
-    if (chunk_sq == 0) continue;
-    prm.out = static_cast<uint16_t*>(out->ptr);
-    prm.out_ss = out->stride_s;
-    prm.out_sh = out->stride_h;
-    prm.group = Hq / Hkv;
-    prm.scale_log2 = scale * 1.4426950408889634f;
-    prm.status = info->status;
-    prm.wait_limit_ns = g_wait_limit_ns;
-    prm.test_stall = g_test_stall;
-    const int n_qtiles = (chunk_sq + skattn::kRowsPerCta - 1) / skattn::kRowsPerCta;
-    st = (D == 64) ? launch_attn<64>(prm, n_qtiles, Hq, nb, stream, info)
-                   : launch_attn<128>(prm, n_qtiles, Hq, nb, stream, info);
-    if (st != SK_OK) return st;
-  }
-  return SK_OK;
+  return varlen_persistent(q, k, v, cu_q, cu_k, used_q, used_k, nseg, Hq, Hkv, scale, out, D, stream, info);
 }
 
 }  // namespace
@@ -855,15 +766,5 @@ sk_status_t sk_test_stall_mma(int32_t on) {
 }
 
 int32_t sk_abi_version(void) { return kAbiVersion; }
-
-// Development hook (not part of the header's interface): selects the
-// attention kernel variant for side-by-side timing.
-SK_API sk_status_t sk_debug_kernel_variant(int32_t v) {
-  if (v < 0 || v > 11) return fail(SK_ERR_INVALID_ARG, "variant must be in 0..11");
-  std::lock_guard<std::mutex> lk(g_mu);
-  g_kernel_variant = v;
-  return SK_OK;
-}
-
 
 }  // extern "C"
