@@ -174,9 +174,10 @@ SK_API sk_status_t attn_fwd_split_kv_scatter(const sk_tensor_t* q, const sk_tens
  *   out  [1, Tq, num_q_heads, head_dim] (written on the segments' rows only;
  *        rows outside every segment are not touched); must not overlap the
  *        inputs or itself.
- * A segment with no valid key writes zeros.  One kernel launch per 8
- * segments, on `stream`.  Returns SK_OK, SK_ERR_INVALID_ARG,
- * SK_ERR_UNSUPPORTED or SK_ERR_CUDA.
+ * A segment with no valid key writes zeros.  One kernel launch per 1024
+ * segments (the segments of a launch are processed longest first), on
+ * `stream`.  Returns SK_OK, SK_ERR_INVALID_ARG, SK_ERR_UNSUPPORTED or
+ * SK_ERR_CUDA.
  */
 SK_API sk_status_t attn_fwd_varlen(const sk_tensor_t* q, const sk_tensor_t* k, const sk_tensor_t* v,
                                    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
@@ -215,7 +216,7 @@ SK_API sk_status_t attn_fwd_varlen(const sk_tensor_t* q, const sk_tensor_t* k, c
  *              final roundings); dims past rot_dim within one ulp of y.
  *              1: return exactly the bits of that exact evaluation (fp32 with
  *              an error bound, elements the bound cannot decide redone in
- *              fp64), about 2.5 times slower.
+ *              fp64), about twice as slow.
  * Returns SK_OK, SK_ERR_INVALID_ARG, SK_ERR_UNSUPPORTED or SK_ERR_CUDA.
  */
 SK_API sk_status_t qk_rmsnorm_rope(const sk_tensor_t* q, const sk_tensor_t* k, const void* w_q,
