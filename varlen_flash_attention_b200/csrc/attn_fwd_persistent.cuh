@@ -26,14 +26,16 @@
 //              of its own score row, and at the end of a unit reads O, divides
 //              by the row sum and stores the bf16 row.
 //   warp 8     TMA producer: Q tiles per unit, K and V tiles into rings.
-//   warp 9     TMEM allocator and tcgen05.mma issuer.
+//   warp 9     TMEM allocator and tcgen05.mma issuer.  Per KV tile j the
+//              order is PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), each PV in two
+//              halves (keys 0-63 once the softmax has released them, then
+//              keys 64-127): PV takes P from TMEM (A operand) and V from
+//              shared memory, so only K, V and Q are read from shared memory.
+//              S_X(j+1) overwrites the columns PV_X(j) reads P from; it is
+//              issued behind PV_X(j) on the same in-order MMA pipe, with no
+//              wait in between.
 //   warps 10-11 idle (they complete the third warpgroup, whose registers go
-//              to the softmax warpgroups).  Per KV tile j the
-//              order is PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): PV takes P from
-//              TMEM (A operand) and V from shared memory, so only K, V and Q
-//              are read from shared memory.  S_X(j+1) overwrites the columns
-//              PV_X(j) reads P from; it is issued behind PV_X(j) on the same
-//              in-order MMA pipe, with no wait in between.
+//              to the softmax warpgroups).
 // TMEM (512 columns): S_A/P_A [0,128), S_B/P_B [128,256), O_A [256,256+D),
 // O_B [384,384+D).
 // Every wait is bounded (globaltimer); on expiry the CTA raises the device
@@ -71,7 +73,7 @@ struct PSmemLayout {
   static constexpr uint32_t kQTile = kBlockM * D * 2;
   static constexpr uint32_t kKVTile = kBlockN * D * 2;
   static constexpr int kKS = D == 128 ? 3 : 4;  // K ring depth
-  static constexpr int kVS = D == 128 ? 2 : 4;                 // V ring depth
+  static constexpr int kVS = D == 128 ? 2 : 4;  // V ring depth
   static constexpr uint32_t kQ = 0;                              // + tile * kQTile
   static constexpr uint32_t kK = kQ + kTilesPerCta * kQTile;     // + stage * kKVTile
   static constexpr uint32_t kV = kK + kKS * kKVTile;             // + stage * kKVTile
