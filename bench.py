@@ -246,6 +246,18 @@ def combine_ranks(flop_per_step, steps, dt_ms, dist, device="cuda"):
     return dt_max, total / (dt_max / 1e3) / 1e12
 
 
+def cpu_model():
+    """The host CPU's model name (for the CPU baseline's record)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_oracle_sample(w, gpu_out=None, target_s=10.0, seed=0):
     """Time the fp64 oracle on a bounded row sample of the workload (host cores).
 
@@ -271,7 +283,9 @@ def cpu_oracle_sample(w, gpu_out=None, target_s=10.0, seed=0):
     fl = flops_of(w, rows)
     cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
            "sample": f"{len(rows)} of {w.Sq} query rows x {w.Hq} heads x {w.B} batch rows of {w.name} "
-                     f"({fl / 1e9:.1f} GFLOP, {dt:.1f} s)"}
+                     f"({fl / 1e9:.1f} GFLOP, {dt:.1f} s)",
+           "cpu": cpu_model(),
+           "all_rows_s": flops_of(w) / (fl / dt)}  # linear extrapolation to every valid row
     if gpu_out is None:
         return cpu, None
     got = gpu_out[:, rows].float().cpu().numpy().astype(np.float64)
