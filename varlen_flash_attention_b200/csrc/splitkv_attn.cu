@@ -489,9 +489,11 @@ sk_status_t varlen_persistent(const sk_tensor_t* q, const sk_tensor_t* k, const 
 }
 
 // Packed varlen input: segment i owns query rows [cu_q[i], cu_q[i+1]) and key
-// rows [cu_k[i], cu_k[i+1]) of single-row tensors; each segment becomes one
-// kernel entry whose tensor maps start at the segment's first row (no prefix,
-// the segment's keys are the suffix), so the block-diagonal mask costs nothing.
+// rows [cu_k[i], cu_k[i+1]) of single-row tensors.  Validation here; the launch
+// (varlen_persistent) uses one tensor map per packed tensor and passes each
+// segment's first rows and lengths in the launch parameters, so the
+// block-diagonal mask costs nothing: a unit only ever loads its own segment's
+// rows.
 sk_status_t varlen_impl(const sk_tensor_t* q, const sk_tensor_t* k, const sk_tensor_t* v,
                         const int32_t* cu_q, const int32_t* cu_k, const int32_t* used_q,
                         const int32_t* used_k, int32_t nseg, int32_t Hq, int32_t Hkv, float scale,
