@@ -24,7 +24,10 @@
 //              running max raised only past kRescaleLog2, then O rescaled in
 //              TMEM), writes P as bf16 pairs back over the first 64 columns
 //              of its own score row, and at the end of a unit reads O, divides
-//              by the row sum and stores the bf16 row.
+//              by the row sum and stores the bf16 row.  After a unit's first
+//              tile the row is loaded in two halves and the first half's
+//              exponentials run on the running max while the second half
+//              arrives; the tile's max is checked before any key is released.
 //   warp 8     TMA producer: Q tiles per unit, K and V tiles into rings.
 //   warp 9     TMEM allocator and tcgen05.mma issuer.  Per KV tile j the
 //              order is PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), each PV in two
@@ -196,6 +199,19 @@ __device__ __forceinline__ uint16_t* unit_row_ptr(const VarlenParams& p, const P
   return p.out + static_cast<int64_t>(t.q_off + row) * p.out_ss + static_cast<int64_t>(t.hq) * p.out_sh;
 }
 
+// Maximum of 64 scores s[B .. B + 63]: two chains of three-input maxima.
+template <int B>
+__device__ __forceinline__ float half_max(const float (&s)[kBlockN]) {
+  float mx[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    mx[k] = fmaxf(s[B + k], s[B + k + 2]);
+#pragma unroll
+    for (int c = B + 4 + k; c < B + 64; c += 4) mx[k] = skptx::fmax3(mx[k], s[c], s[c + 2]);
+  }
+  return fmaxf(mx[0], mx[1]);
+}
+
 // Columns [32 * C, 32 * C + 32) of one score row (already masked) -> 16 bf16
 // pairs of p = 2^(s * sl2 - m) in pk, their fp32 sum added to acc.  Masked
 // columns (partial tile) are exact zeros.
@@ -253,18 +269,73 @@ __device__ __forceinline__ float exp_row_release(const float (&s)[kBlockN], floa
   return a0 + a1;
 }
 
-// Maximum of 64 scores s[B .. B + 63]: two chains of three-input maxima.
-template <int B>
-__device__ __forceinline__ float half_max(const float (&s)[kBlockN]) {
-  float mx[2];
+// Tiles after the first, scores loaded in two halves: the exponentials of keys
+// 0-63 run on the running maximum m while keys 64-127 are still on their way
+// from TMEM; the tile's own maximum is checked before anything is released.
+// Returns false (nothing released, stores may be in flight) when some row of
+// the warp needs m raised by more than 2^kRescaleLog2: s then holds the whole
+// masked row for the regular path.  Otherwise the same P and sum as
+// exp_row_release with the same m.
+template <bool kPartial>
+__device__ __forceinline__ bool exp_row_split_load(float (&s)[kBlockN], uint32_t tS, float sl2, float m, int nvalid,
+                                                   uint32_t bar_lo, uint32_t bar_hi, float& sum) {
+  {
+    uint32_t u[2][32];
+    skptx::tmem_ld32(tS, u[0]);
+    skptx::tmem_ld32(tS + 32, u[1]);
+    skptx::tmem_wait_ld();
+    skptx::reg_fence(u[0]);
+    skptx::reg_fence(u[1]);
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    mx[k] = fmaxf(s[B + k], s[B + k + 2]);
-#pragma unroll
-    for (int c = B + 4 + k; c < B + 64; c += 4) mx[k] = skptx::fmax3(mx[k], s[c], s[c + 2]);
+    for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(u[c / 32][c % 32]);
   }
-  return fmaxf(mx[0], mx[1]);
+  uint32_t w[2][32];
+  skptx::tmem_ld32(tS + 64, w[0]);  // in flight during the first exponentials
+  skptx::tmem_ld32(tS + 96, w[1]);
+  if (kPartial) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+      if (c >= nvalid) s[c] = -INFINITY;
+  }
+  const uint64_t sl2_2 = skptx::f2_pack(sl2, sl2);
+  const uint64_t negm_2 = skptx::f2_pack(-m, -m);
+  uint64_t acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = 0;
+  uint32_t pa[16], pb[16];
+  exp_chunk<kPartial, 0>(s, sl2_2, negm_2, nvalid, pa, acc);
+  skptx::tmem_st16(tS, pa);
+  exp_chunk<kPartial, 1>(s, sl2_2, negm_2, nvalid, pb, acc);
+  skptx::tmem_st16(tS + 16, pb);
+  skptx::tmem_wait_ld();
+  skptx::reg_fence(w[0]);
+  skptx::reg_fence(w[1]);
+#pragma unroll
+  for (int c = 64; c < kBlockN; ++c) s[c] = __uint_as_float(w[(c - 64) / 32][c % 32]);
+  if (kPartial) {
+#pragma unroll
+    for (int c = 64; c < kBlockN; ++c)
+      if (c >= nvalid) s[c] = -INFINITY;
+  }
+  const float mt = fmaxf(half_max<0>(s), half_max<64>(s)) * sl2;
+  if (__any_sync(0xffffffffu, mt > m + kRescaleLog2)) return false;
+  exp_chunk<kPartial, 2>(s, sl2_2, negm_2, nvalid, pa, acc);
+  skptx::tmem_wait_st();
+  skptx::tc_fence_before();
+  skptx::mbar_arrive(bar_lo);
+  skptx::tmem_st16(tS + 32, pa);
+  exp_chunk<kPartial, 3>(s, sl2_2, negm_2, nvalid, pb, acc);
+  skptx::tmem_st16(tS + 48, pb);
+  skptx::tmem_wait_st();
+  skptx::tc_fence_before();
+  skptx::mbar_arrive(bar_hi);
+  const uint64_t a = skptx::add2(skptx::add2(acc[0], acc[1]), skptx::add2(acc[2], acc[3]));
+  float a0, a1;
+  skptx::f2_unpack(a, a0, a1);
+  sum = a0 + a1;
+  return true;
 }
+
 
 // S = Q K^T: 128 x 128 x D, both operands K-major in shared memory
 // (64-column sub-tiles kSub bytes apart).  Warp-collective.
@@ -526,7 +597,17 @@ __device__ __forceinline__ void softmax_rows(const Params& p, const PCtx<D>& cx,
       const int nvalid = tile_valid(j, t.tP, t.nkp, t.nks);
       const bool partial = nvalid < kBlockN;
       float s[kBlockN];
-      {
+      if (j > 0) {  // the common case: exponentials start on the running max
+        float sum;
+        const bool done =
+            partial ? exp_row_split_load<true>(s, tS_, sl2, m_run, nvalid, bar(L::bPLo + x), bar(L::bPHi + x), sum)
+                    : exp_row_split_load<false>(s, tS_, sl2, m_run, nvalid, bar(L::bPLo + x), bar(L::bPHi + x), sum);
+        if (done) {
+          l_run += sum;
+          continue;
+        }
+        skptx::tmem_wait_st();  // the early P stores land before they are overwritten
+      } else {  // first tile of the unit: its maximum starts the running max
         uint32_t uu[4][32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) skptx::tmem_ld32(tS_ + c * 32, uu[c]);
@@ -536,7 +617,7 @@ __device__ __forceinline__ void softmax_rows(const Params& p, const PCtx<D>& cx,
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(uu[c / 32][c % 32]);
       }
-      if (partial) {
+      if (partial && j == 0) {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
           if (c >= nvalid) s[c] = -INFINITY;
