@@ -194,3 +194,20 @@ def test_nan_rows_sharing_the_last_key_tile(sk):
     assert np.all(np.isfinite(got))
     _compare(got, ref, "NaN/Inf pad keys in the last tile")
     assert sk.sk_device_status() == 0
+
+
+def test_varlen_repeated_calls_bitwise_identical(sk):
+    """64 unequal segments: repeated calls give identical bits (each row is
+    written once, by the thread that owns it)."""
+    g = torch.Generator().manual_seed(31)
+    lens = torch.randint(1, 900, (64,), generator=g).tolist()
+    q, k, v, cq, ck = _packed(31, lens, lens, 4, 2, 128)
+    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    first = sk.attn_fwd_varlen(dq, dk, dv, cq, ck)
+    out = torch.full_like(first, float("nan"))
+    for _ in range(3):
+        sk.attn_fwd_varlen(dq, dk, dv, cq, ck, out=out)
+        torch.cuda.synchronize()
+        assert torch.equal(first.view(torch.int16), out.view(torch.int16))
+        out.fill_(float("nan"))
+    assert sk.sk_device_status() == 0
