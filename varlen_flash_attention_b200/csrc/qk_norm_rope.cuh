@@ -355,6 +355,13 @@ __global__ void __launch_bounds__(kNormRopeThreads, kNormRopeMinBlocks) qk_norm_
 
 constexpr int kFastThreads = 256;
 
+// 16-byte store with the streaming (evict-first) cache hint: the rewritten
+// rows are not read again by this kernel, so their L2 lines go first.
+__device__ __forceinline__ void st_stream_v4(uint16_t* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 // fp32 instance, one token per warp: 32 / (D/8) rows per load instruction,
 // so a warp streams through its token's heads in contiguous runs (BATCH
 // loads of (32 / (D/8)) consecutive heads per iteration, the next batch in
@@ -485,7 +492,7 @@ __global__ void __launch_bounds__(kFastThreads, MINB) qk_norm_rope_warp_kernel(c
         const float zc = fmaf(bf16_hi(pb[i]), sg[2 * i + 1], bf16_hi(yb[i]) * c[2 * i + 1]);
         zb[i] = rotates ? pack_bf16x2_rn(za, zc) : yb[i];
       }
-      if (h < H) *reinterpret_cast<uint4*>(row_ptr(h)) = make_uint4(zb[0], zb[1], zb[2], zb[3]);
+      if (h < H) st_stream_v4(row_ptr(h), make_uint4(zb[0], zb[1], zb[2], zb[3]));
     }
 #pragma unroll
     for (int j = 0; j < BATCH; ++j) xv[j] = xn[j];
